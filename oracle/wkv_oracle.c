@@ -1,0 +1,194 @@
+/*
+ * fp64 CPU oracle for RWKV's WKV time-mixing operator.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call this
+ * file; only the tests, the smoke check and the benchmark's CPU-baseline leg do. It
+ * shares no code, header or constant with the CUDA library.
+ *
+ * It is written to be checked by eye against the pages, not to be fast: no blocking,
+ * no stabilisation, no reordering. Everything is double precision; exponents are formed
+ * as sums first and exponentiated afterwards.
+ *
+ * Sources (page title, then section):
+ *   [concept]  "RWKV（Receptance Weighted Key Value）概念" (compassingai.com),
+ *              section 3.2 "时间混合（Time-mixing）与 WKV 算子": the wkv_t equation and
+ *              out_t = sigmoid(receptance_t) * wkv_t.
+ *   [notes]    "RWKV - 把 RNN 重新带回 Transformer 时代的线性大模型" (papernotes,
+ *              2023_rwkv): "一句话总结" (the recurrence a_t, b_t and the output that uses
+ *              a_{t-1}, b_{t-1}), "关键设计 2：WKV 算子" (parallel form and RNN cell),
+ *              "关键设计 4：双执行模式" (single-token inference step).
+ *
+ * Layout: k, v, r, y, dy, dk, dv, dr are (B, T, C) row-major (C fastest); w, u, dw, du
+ * are [C]. Time is 0-based here; the pages' t is our t + 1. All functions return 0, or
+ * -1 on a NULL required pointer / negative size / allocation failure.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#define AT(b, t, c) ((((int64_t)(b)) * T + (t)) * C + (c))
+
+static double sigm(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/*
+ * O1: the parallel (summation) form, O(T^2) per channel.
+ * [concept] 3.2 and [notes] "关键设计 2": for 1-based t,
+ *   wkv_t = (sum_{i<t} e^{-(t-1-i)w + k_i} v_i + e^{u + k_t} v_t)
+ *         / (sum_{i<t} e^{-(t-1-i)w + k_i}     + e^{u + k_t})
+ *   y_t   = sigmoid(r_t) * wkv_t            (r == NULL: y_t = wkv_t, no gate)
+ * Optional initial state (A0, B0) [B*C]: the true numerator and denominator of the past
+ * before the first token; it enters token t (0-based) decayed by e^{-t w}, the same
+ * weight the recurrence gives it. NULL means no past.
+ */
+int oracle_wkv_direct(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
+                      const double *k, const double *v, const double *r, double *y,
+                      const double *A0, const double *B0)
+{
+    if (B < 0 || T < 0 || C < 0 || !w || !u || !k || !v || !y) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t c = 0; c < C; ++c)
+            for (int64_t t = 0; t < T; ++t) {
+                double num = 0.0, den = 0.0;
+                if (A0 && B0) {
+                    double e = exp(-(double)t * w[c]);
+                    num += e * A0[b * C + c];
+                    den += e * B0[b * C + c];
+                }
+                for (int64_t i = 0; i < t; ++i) {
+                    double e = exp(-(double)(t - 1 - i) * w[c] + k[AT(b, i, c)]);
+                    num += e * v[AT(b, i, c)];
+                    den += e;
+                }
+                double e = exp(u[c] + k[AT(b, t, c)]);
+                num += e * v[AT(b, t, c)];
+                den += e;
+                double wkv = num / den;
+                y[AT(b, t, c)] = r ? sigm(r[AT(b, t, c)]) * wkv : wkv;
+            }
+    return 0;
+}
+
+/*
+ * O2: the recurrent form, unstabilised.
+ * [notes] "一句话总结": a_t = e^{-w} a_{t-1} + e^{k_t} v_t, b_t = e^{-w} b_{t-1} + e^{k_t},
+ * and the output at t uses the state before the token:
+ *   wkv_t = (a_{t-1} + e^{u+k_t} v_t) / (b_{t-1} + e^{u+k_t}).
+ * State in (A0, B0) and out (A1, B1) are the true (unscaled) numerator and denominator,
+ * [B*C] each; NULL in means a_0 = b_0 = 0, NULL out means not wanted.
+ */
+int oracle_wkv_recurrent(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
+                         const double *k, const double *v, const double *r, double *y,
+                         const double *A0, const double *B0, double *A1, double *B1)
+{
+    if (B < 0 || T < 0 || C < 0 || !w || !u || !k || !v || !y) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t c = 0; c < C; ++c) {
+            double a = (A0 && B0) ? A0[b * C + c] : 0.0;
+            double d = (A0 && B0) ? B0[b * C + c] : 0.0;
+            double decay = exp(-w[c]);
+            for (int64_t t = 0; t < T; ++t) {
+                double kt = k[AT(b, t, c)], vt = v[AT(b, t, c)];
+                double cur = exp(u[c] + kt);
+                double wkv = (a + cur * vt) / (d + cur);
+                y[AT(b, t, c)] = r ? sigm(r[AT(b, t, c)]) * wkv : wkv;
+                double ek = exp(kt);
+                a = decay * a + ek * vt;
+                d = decay * d + ek;
+            }
+            if (A1) A1[b * C + c] = a;
+            if (B1) B1[b * C + c] = d;
+        }
+    return 0;
+}
+
+/*
+ * Single-token step for N sequences x L layers, state updated in place.
+ * [notes] "关键设计 4" (inference keeps only the numerator/denominator state and updates
+ * it once per token) with the WKV lines of "一句话总结". Layer l of sequence n uses
+ * w[l*C + c], u[l*C + c]. k, v, r, y, A, Bd are [N, L, C]; A, Bd are true (unscaled).
+ */
+int oracle_wkv_decode(int64_t N, int64_t L, int64_t C, const double *w, const double *u,
+                      const double *k, const double *v, const double *r, double *y,
+                      double *A, double *Bd)
+{
+    if (N < 0 || L < 0 || C < 0 || !w || !u || !k || !v || !y || !A || !Bd) return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t l = 0; l < L; ++l)
+            for (int64_t c = 0; c < C; ++c) {
+                int64_t s = (n * L + l) * C + c, p = l * C + c;
+                double cur = exp(u[p] + k[s]);
+                double wkv = (A[s] + cur * v[s]) / (Bd[s] + cur);
+                y[s] = r ? sigm(r[s]) * wkv : wkv;
+                double ek = exp(k[s]);
+                A[s] = exp(-w[p]) * A[s] + ek * v[s];
+                Bd[s] = exp(-w[p]) * Bd[s] + ek;
+            }
+    return 0;
+}
+
+/*
+ * O4: gradients of L = sum_t dy_t . y_t with respect to k, v, w, u (and r), analytic.
+ * The pages say only that the operator supports ordinary backpropagation; the formulas
+ * below are derived from the parallel form of [concept] 3.2 by the chain rule.
+ * With N_t, D_t the numerator and denominator of wkv_t, g_t = dy_t sigmoid(r_t) and
+ * h_t = g_t / D_t (0-based, sums over t > i):
+ *   beta_i   = sum h_t e^{-(t-1-i)w},          gamma_i   = sum h_t wkv_t e^{-(t-1-i)w}
+ *   betad_i  = sum (t-1-i) h_t e^{-(t-1-i)w},  gammad_i  = sum (t-1-i) h_t wkv_t e^{-(t-1-i)w}
+ *   dv_i = e^{k_i} (h_i e^u + beta_i)
+ *   dk_i = e^{k_i} (h_i e^u (v_i - wkv_i) + v_i beta_i - gamma_i)
+ *   dw   = -sum_{b,i} e^{k_i} (v_i betad_i - gammad_i)      (w is the positive decay rate)
+ *   du   =  sum_{b,t} h_t e^{u+k_t} (v_t - wkv_t)
+ *   dr_t = dy_t wkv_t sigmoid(r_t) (1 - sigmoid(r_t))
+ * computed by the reverse recurrences beta_{i-1} = h_i + e^{-w} beta_i and
+ * betad_{i-1} = e^{-w} (betad_i + beta_i) (and the same for gamma).
+ * r == NULL: no gate (g_t = dy_t) and dr is not written. dr may be NULL.
+ * dw, du [C] are overwritten with the sums over b and t.
+ */
+int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
+                        const double *k, const double *v, const double *r, const double *dy,
+                        double *dk, double *dv, double *dw, double *du, double *dr)
+{
+    if (B < 0 || T < 0 || C < 0 || !w || !u || !k || !v || !dy || !dk || !dv || !dw || !du)
+        return -1;
+    double *wkv = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    double *D = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (!wkv || !D) { free(wkv); free(D); return -1; }
+    for (int64_t c = 0; c < C; ++c) { dw[c] = 0.0; du[c] = 0.0; }
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t c = 0; c < C; ++c) {
+            double decay = exp(-w[c]), eu = exp(u[c]);
+            double a = 0.0, d = 0.0;
+            for (int64_t t = 0; t < T; ++t) {                /* forward, as O2 */
+                double kt = k[AT(b, t, c)], vt = v[AT(b, t, c)];
+                double cur = exp(u[c] + kt);
+                D[t] = d + cur;
+                wkv[t] = (a + cur * vt) / D[t];
+                double ek = exp(kt);
+                a = decay * a + ek * vt;
+                d = decay * d + ek;
+            }
+            double beta = 0.0, gamma = 0.0, betad = 0.0, gammad = 0.0;
+            double dwc = 0.0, duc = 0.0;
+            for (int64_t i = T - 1; i >= 0; --i) {           /* reverse */
+                double ki = k[AT(b, i, c)], vi = v[AT(b, i, c)], dyi = dy[AT(b, i, c)];
+                double s = r ? sigm(r[AT(b, i, c)]) : 1.0;
+                double h = dyi * s / D[i];
+                double ek = exp(ki);
+                dv[AT(b, i, c)] = ek * (h * eu + beta);
+                dk[AT(b, i, c)] = ek * (h * eu * (vi - wkv[i]) + vi * beta - gamma);
+                dwc += -ek * (vi * betad - gammad);
+                duc += h * eu * ek * (vi - wkv[i]);
+                if (r && dr) dr[AT(b, i, c)] = dyi * wkv[i] * s * (1.0 - s);
+                betad = decay * (betad + beta);
+                gammad = decay * (gammad + gamma);
+                beta = h + decay * beta;
+                gamma = h * wkv[i] + decay * gamma;
+            }
+            dw[c] += dwc;
+            du[c] += duc;
+        }
+    free(wkv);
+    free(D);
+    return 0;
+}

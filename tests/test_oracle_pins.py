@@ -1,0 +1,258 @@
+"""Pins for the fp64 oracle: each test ties it to something other than itself.
+
+The pages print no worked numeric example, so the oracle is pinned by: two independent
+forms of the same definition (parallel sum vs recurrence), a textbook library route
+(SciPy softmax), closed forms for special cases, exact rational arithmetic, invariants
+(a convex combination stays within the range of its points) and finite differences.
+A plausible slip in the oracle (a dropped current-token term, a decay that starts one
+step early or late, a sign of w, u on the wrong term, a transposed index, a wrong
+gradient accumulator order) fails at least one of these.
+"""
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+import wkv_inputs
+
+
+def _rand(B, T, C, seed, k_std=1.0, logw=(-3.0, 1.0)):
+    g = np.random.Generator(np.random.PCG64(seed))
+    w = np.exp(g.uniform(*logw, size=C))
+    u = g.uniform(-1, 1, size=C)
+    k = g.normal(0, k_std, size=(B, T, C))
+    v = g.standard_normal((B, T, C))
+    r = g.standard_normal((B, T, C))
+    return w, u, k, v, r
+
+
+def test_parallel_form_equals_recurrence():
+    # "关键设计 2" gives both forms of the same operator.
+    w, u, k, v, r = _rand(3, 40, 7, 1)
+    y1 = oracle.wkv_direct(w, u, k, v, r)
+    y2 = oracle.wkv_recurrent(w, u, k, v, r)
+    np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-13)
+
+
+def test_parallel_form_equals_recurrence_with_initial_state():
+    w, u, k, v, r = _rand(2, 25, 5, 2)
+    g = np.random.Generator(np.random.PCG64(3))
+    A0 = g.standard_normal((2, 5)) * 3.0
+    B0 = g.uniform(0.5, 4.0, size=(2, 5))
+    y1 = oracle.wkv_direct(w, u, k, v, r, A0, B0)
+    y2 = oracle.wkv_recurrent(w, u, k, v, r, A0, B0)
+    np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-13)
+
+
+def test_matches_scipy_softmax_route():
+    # The operator as causal attention with logits k_i - (t-1-i)w and u + k_t.
+    w, u, k, v, _ = _rand(1, 12, 4, 4, k_std=2.0)
+    ys = oracle.wkv_softmax_form(w, u, k[0], v[0])
+    yd = oracle.wkv_direct(w, u, k, v)[0]
+    np.testing.assert_allclose(yd, ys, rtol=1e-12, atol=1e-13)
+
+
+def test_single_token_gives_v():
+    w, u, k, v, _ = _rand(4, 1, 9, 5, k_std=5.0)
+    for f in (oracle.wkv_direct, oracle.wkv_recurrent):
+        np.testing.assert_allclose(f(w, u, k, v), v, rtol=1e-15, atol=0)
+
+
+def test_constant_value_is_reproduced():
+    w, u, k, _, _ = _rand(2, 30, 6, 6, k_std=3.0)
+    v = np.broadcast_to(np.linspace(-2, 2, 6), (2, 30, 6)).copy()
+    for f in (oracle.wkv_direct, oracle.wkv_recurrent):
+        np.testing.assert_allclose(f(w, u, k, v), v, rtol=1e-14, atol=1e-15)
+
+
+def test_output_within_prefix_range():
+    w, u, k, v, _ = _rand(2, 50, 8, 7, k_std=3.0)
+    y = oracle.wkv_recurrent(w, u, k, v)
+    lo = np.minimum.accumulate(v, axis=1)
+    hi = np.maximum.accumulate(v, axis=1)
+    eps = 1e-12
+    assert np.all(y >= lo - eps) and np.all(y <= hi + eps)
+
+
+def test_gate_multiplies_by_sigmoid():
+    w, u, k, v, r = _rand(1, 10, 3, 8)
+    np.testing.assert_allclose(oracle.wkv_direct(w, u, k, v, r),
+                               oracle.wkv_direct(w, u, k, v) / (1 + np.exp(-r)), rtol=1e-14)
+
+
+def test_fast_decay_leaves_last_two_tokens():
+    # w -> large: every token older than i = t-1 is forgotten (the most recent past token
+    # is not decayed: exponent -(t-1-i)w is zero for i = t-1).
+    _, u, k, v, _ = _rand(2, 20, 5, 9)
+    w = np.full(5, 80.0)
+    y = oracle.wkv_recurrent(w, u, k, v)
+    ek_prev, ecur = np.exp(k[:, :-1]), np.exp(u + k[:, 1:])
+    want = (ek_prev * v[:, :-1] + ecur * v[:, 1:]) / (ek_prev + ecur)
+    np.testing.assert_allclose(y[:, 1:], want, rtol=1e-13)
+    np.testing.assert_allclose(y[:, 0], v[:, 0], rtol=1e-15)
+
+
+def test_huge_bonus_gives_current_value():
+    w, _, k, v, _ = _rand(1, 15, 4, 10)
+    u = np.full(4, 60.0)
+    np.testing.assert_allclose(oracle.wkv_direct(w, u, k, v), v, rtol=1e-12, atol=1e-12)
+
+
+def test_no_decay_is_prefix_weighted_mean():
+    # w -> 0: a softmax-weighted mean over the whole prefix, by cumulative sums.
+    _, u, k, v, _ = _rand(2, 30, 3, 11)
+    w = np.full(3, 1e-14)
+    y = oracle.wkv_direct(w, u, k, v)
+    ek = np.exp(k)
+    past_num = np.cumsum(ek * v, axis=1) - ek * v
+    past_den = np.cumsum(ek, axis=1) - ek
+    cur = np.exp(u + k)
+    want = (past_num + cur * v) / (past_den + cur)
+    np.testing.assert_allclose(y, want, rtol=1e-11)
+
+
+@pytest.mark.parametrize("j", [0, 3, 9])
+def test_geometric_closed_form(j):
+    # k constant and v a unit impulse at token j: the weights are a geometric sequence.
+    T, C = 14, 3
+    w = np.array([0.05, 0.7, 2.5])
+    u = np.array([-0.4, 0.3, 1.1])
+    k = np.full((1, T, C), 1.7)
+    v = np.zeros((1, T, C))
+    v[0, j, :] = 1.0
+    y = oracle.wkv_recurrent(w, u, k, v)[0]
+    for t in range(T):                      # 0-based t; token t has t past tokens
+        past = (1 - np.exp(-t * w)) / (1 - np.exp(-w))   # sum_{m=0}^{t-1} e^{-m w}
+        den = past + np.exp(u)
+        if t < j:
+            want = np.zeros(C)
+        elif t == j:
+            want = np.exp(u) / den
+        else:
+            want = np.exp(-(t - 1 - j) * w) / den
+        np.testing.assert_allclose(y[t], want, rtol=1e-12, atol=1e-15)
+
+
+def test_exact_rational_example():
+    # e^{-w} = 1/2, e^{u} = 3, e^{k_i} = i + 1: every weight is rational.
+    T = 7
+    vs = [3, -1, 4, 1, -5, 9, 2]
+    half = Fraction(1, 2)
+    want = []
+    for t in range(T):
+        num = sum(half ** (t - 1 - i) * (i + 1) * vs[i] for i in range(t))
+        den = sum(half ** (t - 1 - i) * (i + 1) for i in range(t))
+        num += 3 * (t + 1) * vs[t]
+        den += 3 * (t + 1)
+        want.append(num / den)
+    w = np.array([math.log(2.0)])
+    u = np.array([math.log(3.0)])
+    k = np.log(np.arange(1, T + 1, dtype=np.float64)).reshape(1, T, 1)
+    v = np.array(vs, dtype=np.float64).reshape(1, T, 1)
+    for f in (oracle.wkv_direct, oracle.wkv_recurrent):
+        y = f(w, u, k, v)[0, :, 0]
+        np.testing.assert_allclose(y, [float(q) for q in want], rtol=1e-14)
+
+
+def test_split_invariance_of_state():
+    # Encoding a sequence in two segments and handing the state over gives the same
+    # output and final state as one pass.
+    w, u, k, v, r = _rand(2, 33, 4, 12)
+    y, A, Bd = oracle.wkv_recurrent(w, u, k, v, r, want_state=True)
+    y1, A1, B1 = oracle.wkv_recurrent(w, u, k[:, :20], v[:, :20], r[:, :20], want_state=True)
+    y2 = oracle.wkv_direct(w, u, k[:, 20:], v[:, 20:], r[:, 20:], A1, B1)
+    _, A2, B2 = oracle.wkv_recurrent(w, u, k[:, 20:], v[:, 20:], r[:, 20:], A1, B1,
+                                     want_state=True)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(A2, A, rtol=1e-12)
+    np.testing.assert_allclose(B2, Bd, rtol=1e-12)
+
+
+def test_decode_steps_reproduce_forward():
+    w, u, k, v, r = _rand(3, 12, 5, 13)
+    y = oracle.wkv_direct(w, u, k, v, r)
+    A = np.zeros((3, 1, 5))
+    Bd = np.zeros((3, 1, 5))
+    for t in range(12):
+        yt, A, Bd = oracle.wkv_decode(w[None], u[None], k[:, t:t + 1], v[:, t:t + 1],
+                                      r[:, t:t + 1], A, Bd)
+        np.testing.assert_allclose(yt[:, 0], y[:, t], rtol=1e-12, atol=1e-13)
+
+
+def test_decode_matches_single_step_restatement():
+    d = wkv_inputs.decode_batch(seed=3, N=4, L=3, C=8)
+    A, Bd = oracle.state_from_scaled(d.a, d.b, d.p)
+    k, v, r = d.step(0)
+    y, A1, B1 = oracle.wkv_decode(d.w, d.u, k, v, None, A, Bd)
+    for n in range(4):
+        for l in range(3):
+            yy, (na, nb) = oracle.wkv_single_step(d.w[l], d.u[l], k[n, l], v[n, l],
+                                                  (A[n, l], Bd[n, l]))
+            np.testing.assert_allclose(y[n, l], yy, rtol=1e-13)
+            np.testing.assert_allclose(A1[n, l], na, rtol=1e-13)
+            np.testing.assert_allclose(B1[n, l], nb, rtol=1e-13)
+
+
+def _loss(w, u, k, v, r, dy):
+    return float(np.sum(oracle.wkv_direct(w, u, k, v, r) * dy))
+
+
+@pytest.mark.parametrize("gate", [True, False])
+def test_backward_matches_central_differences(gate):
+    B, T, C = 2, 8, 3
+    w, u, k, v, r = _rand(B, T, C, 14)
+    if not gate:
+        r = None
+    dy = np.random.Generator(np.random.PCG64(15)).standard_normal((B, T, C))
+    g = oracle.wkv_backward(w, u, k, v, r, dy)
+    h = 1e-6
+
+    def fd(name, arr, idx):
+        plus = {"w": w, "u": u, "k": k, "v": v, "r": r}
+        a1 = arr.copy(); a1[idx] += h
+        a2 = arr.copy(); a2[idx] -= h
+        plus[name] = a1
+        lp = _loss(plus["w"], plus["u"], plus["k"], plus["v"], plus["r"], dy)
+        plus[name] = a2
+        lm = _loss(plus["w"], plus["u"], plus["k"], plus["v"], plus["r"], dy)
+        return (lp - lm) / (2 * h)
+
+    for name, arr, grad in (("k", k, g["dk"]), ("v", v, g["dv"])):
+        for idx in np.ndindex(arr.shape):
+            assert fd(name, arr, idx) == pytest.approx(grad[idx], rel=1e-6, abs=1e-8), \
+                (name, idx)
+    for name, arr, grad in (("w", w, g["dw"]), ("u", u, g["du"])):
+        for c in range(C):
+            assert fd(name, arr, (c,)) == pytest.approx(grad[c], rel=1e-6, abs=1e-8), \
+                (name, c)
+    if gate:
+        for idx in np.ndindex(r.shape):
+            assert fd("r", r, idx) == pytest.approx(g["dr"][idx], rel=1e-6, abs=1e-8)
+    else:
+        assert g["dr"] is None
+
+
+def test_spike_inputs_stay_finite_and_in_range():
+    # The bf16 workload's k has entries of +60: e^{62} is far inside fp64's range.
+    x = wkv_inputs.long_bf16(seed=0, B=1, T=256, C=64)
+    y = oracle.wkv_recurrent(x.w, x.u, x.k, x.v)
+    assert np.all(np.isfinite(y))
+    lo = np.minimum.accumulate(x.v.astype(np.float64), axis=1)
+    hi = np.maximum.accumulate(x.v.astype(np.float64), axis=1)
+    assert np.all(y >= lo - 1e-12) and np.all(y <= hi + 1e-12)
+    yd = oracle.wkv_direct(x.w, x.u, x.k[:, :64], x.v[:, :64])
+    np.testing.assert_allclose(yd, y[:, :64], rtol=1e-12, atol=1e-13)
+
+
+def test_golden_fixture_regression():
+    # Values written by tests/golden/make_golden.py from the oracle; keeps the oracle
+    # from drifting between commits.
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "tiny_forward_seed0.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    x = wkv_inputs.tiny_forward(seed=0)
+    y = oracle.wkv_direct(x.w, x.u, x.k, x.v, x.r)
+    for b, t, c, val in rows:
+        assert y[int(b), int(t), int(c)] == pytest.approx(float(val), rel=1e-13, abs=1e-15)
