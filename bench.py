@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""Benchmark of the WKV forward on one batch of the 7B-shaped bf16 workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one wkv_forward_bf16 call over B=8, T=4096, C=4096 (k, v, r, y bf16; fp32
+arithmetic; w = exp(U(-6,2)), u ~ U(-2,2), k ~ N(0,3) with 0.1% set to +60, v, r ~ N(0,1);
+seeded synthetic inputs, see wkv_inputs.py). Inputs (805 MB) and output (268 MB) are
+far larger than the 126 MB L2, so no flush is needed between steps.
+
+Under torchrun (N > 1) every rank runs its own batch (seed = rank) with no collective on
+the data path: weak scaling. Timing: CUDA events on the launching stream, barrier and
+synchronize on both sides, max over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (single thread) on bounded samples of the
+same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "WKV fwd G(B·T·C)/s and HBM GB/s vs B200 peak at B=8,T=4096,C=4096"
+UNIT = "G(B·T·C)/s"
+B, T, C = 8, 4096, 4096
+ELEMS = B * T * C
+BYTES_PER_ELEM = 8          # read k, v, r and write y, 2 bytes each
+FALLBACK_HBM_GBS = 6650.0
+KERNEL = "wkv_fwd_tma_kernel<bf16, gate>"
+KERNEL_SOURCES = ["rwkv_linear_attention_wkv_b200/csrc/wkv_fwd.cu",
+                  "rwkv_linear_attention_wkv_b200/csrc/wkv_step.cuh",
+                  "rwkv_linear_attention_wkv_b200/csrc/wkv_device.cuh"]
+TRAFFIC_FILE = "profiles/wkv_fwd_tma_bf16__B8_T4096_C4096.md"
+
+
+def kernel_digest() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel sources as they are now; else None."""
+    path = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            key, _, val = line.strip()[2:].partition(":")
+            fields[key.strip()] = val.strip().strip("`")
+    try:
+        if fields.get("source_digest") != kernel_digest():
+            return None
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_indices):
+        self.gpu_indices = gpu_indices
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    idx = int(parts[0])
+                    sm, smax = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                if self.gpu_indices is not None and idx not in self.gpu_indices:
+                    continue
+                rows.append((sm, smax, parts[5:9]))
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, _, flags in rows for n, f in zip(names, flags)
+                          if f.lower().startswith("active")})
+        loaded = [r for r in rows if r[0] > 0.5 * r[1]] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def visible_gpu_indices(n):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return [int(x) for x in vis.split(",")][:n]
+        except ValueError:
+            return None
+    return list(range(n))
+
+
+def cpu_oracle_rate(x, budget_s=10.0, max_rows=None):
+    """fp64 recurrence oracle over whole batch rows of the workload until the budget is
+    spent (at least one row). Returns (elements per second, rows done)."""
+    import oracle
+    rows = 0
+    t0 = time.perf_counter()
+    nmax = x.B if max_rows is None else min(max_rows, x.B)
+    while rows < nmax:
+        oracle.wkv_recurrent(x.w, x.u, x.k[rows:rows + 1], x.v[rows:rows + 1],
+                             x.r[rows:rows + 1])
+        rows += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return rows * x.T * x.C / dt, rows
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on this host's cores (one thread)."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    import wkv_inputs
+    x = wkv_inputs.long_bf16(seed=0, B=1)      # one batch row; steps sample channels of it
+    # Size each step so that warm-up + timed steps take about a minute in total.
+    probe_c = 64
+    t0 = time.perf_counter()
+    oracle.wkv_recurrent(x.w[:probe_c], x.u[:probe_c], x.k[:, :, :probe_c],
+                         x.v[:, :, :probe_c], x.r[:, :, :probe_c])
+    per_chan = (time.perf_counter() - t0) / probe_c
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    nchan = int(max(8, min(x.C, budget / per_chan)))
+    g = np.random.Generator(np.random.PCG64(1))
+    times = []
+    for s in range(args.warmup + args.steps):
+        c0 = int(g.integers(0, x.C - nchan + 1))
+        sl = slice(c0, c0 + nchan)
+        k, v, r = (np.ascontiguousarray(a[:, :, sl]) for a in (x.k, x.v, x.r))
+        t0 = time.perf_counter()
+        oracle.wkv_recurrent(x.w[sl], x.u[sl], k, v, r)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    elems = nchan * x.T
+    total = sum(times)
+    value = elems * len(times) / total / 1e9
+    sample = (f"per step {nchan} channels x {x.T} tokens of batch row 0 of the B=8,T=4096,"
+              f"C=4096 bf16 workload; fp64 recurrence, 1 thread")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "WKV forward, B=8 T=4096 C=4096 (oracle on a sample)",
+                   "B": B, "T": T, "C": C, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import rwkv_linear_attention_wkv_b200 as W
+    import wkv_inputs
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    x = wkv_inputs.long_bf16(seed=rank)
+
+    def to_bf16(bits, pin=False):
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory() if pin else t.to(dev)
+
+    w = torch.from_numpy(x.w).to(dev)
+    u = torch.from_numpy(x.u).to(dev)
+    k, v, r = (to_bf16(x.bits[n]) for n in "kvr")
+    y = torch.empty_like(k)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        W.wkv_forward_bf16(w, u, k, v, r, y=y)
+    if W.wkv_stream_status() != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(visible_gpu_indices(world) if rank == 0 else None)
+    barrier()
+    if rank == 0:
+        sampler.__enter__()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        W.wkv_forward_bf16(w, u, k, v, r, y=y)
+        ends[i].record(stream)
+    barrier()
+    if rank == 0:
+        sampler.__exit__(None, None, None)
+    if W.wkv_stream_status() != 0:
+        raise RuntimeError("device-side error during the timed region")
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    elapsed_ms = starts[0].elapsed_time(ends[-1])
+    if dist is not None:
+        t = torch.tensor([elapsed_ms, statistics.mean(per_launch)], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, launch_ms = float(t[0]), float(t[1])
+    else:
+        launch_ms = statistics.mean(per_launch)
+    value = world * ELEMS * args.steps / (elapsed_ms / 1e3) / 1e9
+
+    # End to end through the public API: pinned host k, v, r -> device, forward, y -> host.
+    e2e_steps = max(3, min(args.steps, 20))
+    hk, hv, hr = (to_bf16(x.bits[n], pin=True) for n in "kvr")
+    hy = torch.empty(hk.shape, dtype=torch.bfloat16).pin_memory()
+    dk, dv, dr, dy_ = (torch.empty_like(k) for _ in range(4))
+
+    def e2e_step():
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dr.copy_(hr, non_blocking=True)
+        W.wkv_forward_bf16(w, u, dk, dv, dr, y=dy_)
+        hy.copy_(dy_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    e2e_value = world * ELEMS * e2e_steps / (e2e_ms / 1e3) / 1e9
+    assert np.array_equal(hy.view(torch.int16).numpy(), y.view(torch.int16).cpu().numpy()), \
+        "end-to-end result differs from the device-resident run"
+
+    if rank != 0:
+        return
+    peak, peak_kind = hbm_peak()
+    achieved = ELEMS * BYTES_PER_ELEM / (launch_ms / 1e3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, rows = cpu_oracle_rate(x, budget_s=10.0)
+        cpu = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{rows} of 8 batch rows ({rows} x 4096 x 4096 elements) of the same "
+                         f"inputs, fp64 recurrence, 1 thread"}
+    clocks = sampler.summary()
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": "WKV forward bf16 in/out, B=8 T=4096 C=4096 (7B-shaped, "
+                               "k spikes of +60), one batch per GPU",
+                   "B": B, "T": T, "C": C, "storage": "bf16", "global_batch": B * world,
+                   "seq_len": T, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs 805 MB + output 268 MB per step > 126 MB L2; no flush",
+                   "kernel": KERNEL},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": measured_traffic(),
+                     "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": ELEMS * BYTES_PER_ELEM,
+                     "launch_ms": launch_ms},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": 3 * ELEMS * 2, "d2h_bytes_per_step": ELEMS * 2,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 runs under torchrun (one process per GPU)")
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+        try:
+            run_ours(args, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+        return
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+/*
+ * wkv.h — C ABI of the B200 (sm_100a) WKV library (libwkv.so).
+ *
+ * The operator is RWKV's WKV time mixing. For every channel (b, c) of a (B, T, C)
+ * sequence batch, with 1-based token index t:
+ *
+ *   wkv_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t} )
+ *   y_t   = sigmoid(r_t) * wkv_t
+ *
+ * (concept page "RWKV（Receptance Weighted Key Value）概念", section 3.2 "时间混合
+ * （Time-mixing）与 WKV 算子": the wkv_t equation and out_t = sigmoid(Receptance_t) wkv_t).
+ * Equivalently (paper notes "RWKV - 把 RNN 重新带回 Transformer 时代的线性大模型",
+ * "一句话总结"), with a_0 = b_0 = 0,
+ *   a_t = e^{-w} a_{t-1} + e^{k_t} v_t,   b_t = e^{-w} b_{t-1} + e^{k_t},
+ *   wkv_t = (a_{t-1} + e^{u+k_t} v_t) / (b_{t-1} + e^{u+k_t}).
+ * w > 0 is the per-channel decay rate (the value itself, not its logarithm) and u the
+ * per-channel bonus of the current token (same section 3.2).
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers are DEVICE pointers owned by the caller; the library keeps none after the
+ *    call returns and allocates nothing it does not free again within the call's stream
+ *    order.
+ *  - Tensors of shape (B, T, C) are dense row-major, C fastest. w and u are fp32 [C]
+ *    (decode: [L, C]). "bf16" buffers hold IEEE bfloat16 values (passed as void*).
+ *  - Sizes are int64. B, T or C == 0 is a valid empty problem (nothing is launched; a
+ *    requested final state is set to the initial state). Negative sizes, null required
+ *    pointers and pointers not aligned to their element size return
+ *    WKV_ERR_INVALID_ARG / WKV_ERR_ALIGNMENT before anything is enqueued.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream). The return value
+ *    covers argument checks and launch errors only. Errors raised on the device (a
+ *    bounded wait that gave up) are reported by wkv_stream_status().
+ *  - Preconditions that are documented, not checked on the device: inputs finite, w > 0,
+ *    state denominators b > 0. The empty state is (a, b, p) = (0, 0, -1e38) (or NULL);
+ *    never pass -inf.
+ *  - Numerics: fp32 accumulation in a log-max-stabilised base-2 form; no exponential
+ *    overflows for any finite input. bf16 outputs are rounded to nearest even.
+ *  - The library uses one GPU: the device current on the calling thread.
+ */
+#ifndef WKV_H_
+#define WKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define WKV_API __attribute__((visibility("default")))
+#else
+#define WKV_API
+#endif
+
+typedef enum wkv_status {
+  WKV_OK = 0,
+  WKV_ERR_INVALID_ARG = 1, /* negative size, null required pointer, bad workspace size */
+  WKV_ERR_ALIGNMENT = 2,   /* a pointer not aligned to its element size                */
+  WKV_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed              */
+  WKV_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (wkv_stream_status)   */
+  WKV_ERR_UNSUPPORTED = 5  /* a size beyond what the kernels index (e.g. T >= 2^31)    */
+} wkv_status;
+
+/* Human-readable name of a status code. Never NULL. */
+WKV_API const char* wkv_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+WKV_API int wkv_version(void);
+
+/*
+ * Forward, fp32. k, v, r, y: fp32 (B, T, C). w, u: fp32 [C].
+ * r == NULL: no receptance gate (y = wkv). y must not alias k, v or r.
+ * Definition: concept page section 3.2 (see the top of this file).
+ */
+WKV_API int wkv_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                        const float* k, const float* v, const float* r, float* y,
+                        cudaStream_t stream);
+
+/*
+ * Forward, bf16 in and out (k, v, r, y bf16 (B, T, C)); w, u and all arithmetic fp32.
+ * Otherwise as wkv_forward.
+ */
+WKV_API int wkv_forward_bf16(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                             const void* k, const void* v, const void* r, void* y,
+                             cudaStream_t stream);
+
+/*
+ * Forward with state in and out, fp32, for streaming and segment-wise encoding (the
+ * research report "RWKV模型深度研究报告", section 4.4.2: encode a long input segment by
+ * segment and carry the state across; the paper notes' "关键设计 4": the inference state
+ * holds numerator, denominator and a stabilising exponent).
+ *
+ * State layout: three fp32 [B, C] arrays (a, b, p) meaning numerator A = a e^p and
+ * denominator B = b e^p of the past (p in natural log). The representation is not unique:
+ * (a e^s, b e^s, p - s) is the same state; compare states by a/b and p + ln b.
+ * a0/b0/p0: initial state, all three NULL = empty state. a1/b1/p1: final state after the
+ * last token, all three NULL = not wanted; they may alias a0/b0/p0.
+ * Running the two halves of a sequence through this call with the state handed over gives
+ * the result of one call over the whole sequence.
+ *
+ * Long sequences with few channels (B*C small) are split into time segments processed in
+ * parallel; the per-segment carries are combined on the device (decoupled look-back with
+ * bounded waits). This path allocates its scratch with cudaMallocAsync on `stream` and
+ * frees it again in stream order.
+ */
+WKV_API int wkv_forward_state(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                              const float* k, const float* v, const float* r, float* y,
+                              const float* a0, const float* b0, const float* p0, float* a1,
+                              float* b1, float* p1, cudaStream_t stream);
+
+/*
+ * One token for N sequences x L layers (recurrent inference; paper notes "关键设计 4",
+ * the single-token step keeps only the state). k, v, r, y: fp32 [N, L, C]; w, u: fp32
+ * [L, C] (layer l of every sequence uses row l); a, b, p: fp32 [N, L, C] state in the
+ * representation of wkv_forward_state, read and updated in place. r == NULL: no gate.
+ * The output uses the state before the token; the state is then advanced by the token.
+ */
+WKV_API int wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, const float* u,
+                            const float* k, const float* v, const float* r, float* y, float* a,
+                            float* b, float* p, cudaStream_t stream);
+
+/*
+ * Query and clear device-side errors. Synchronises `stream`, then returns WKV_ERR_TIMEOUT
+ * if any kernel of this library on the current device gave up a bounded wait since the
+ * last query (the outputs of that call are then undefined), WKV_ERR_CUDA if the stream
+ * reports a CUDA error, else WKV_OK.
+ */
+WKV_API int wkv_stream_status(cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_H_ */

@@ -1,0 +1,39 @@
+/*
+ * wkv_testing.h — test hooks of libwkv.so. Not part of the operator: these entry points
+ * exist so that the library's failure handling can be exercised without faulting a GPU.
+ */
+#ifndef WKV_TESTING_H_
+#define WKV_TESTING_H_
+
+#include <stdint.h>
+
+#include "wkv.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * Runs the chunked forward on a small internal problem (B = 1, C = 32, three time
+ * segments; every input zero) in which segment 0 withholds its published prefix,
+ * so the look-back of the later segments waits on a flag that nothing sets and gives up
+ * after `wait_ns` nanoseconds (bounded wait; no trap, no hang). The kernel still ends and
+ * the next wkv_stream_status(stream) returns WKV_ERR_TIMEOUT, after which the error word
+ * is clear again. Allocates its buffers with cudaMallocAsync on `stream` and frees them in
+ * stream order. Returns the launch status.
+ */
+WKV_API int wkv_testing_lookback_timeout(uint64_t wait_ns, cudaStream_t stream);
+
+/*
+ * Forces the plain (non-TMA) forward kernel for one fp32 / bf16 forward; otherwise as
+ * wkv_forward / wkv_forward_bf16. Lets tests compare the two kernels on the same inputs.
+ */
+WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const float* w,
+                                      const float* u, const void* k, const void* v,
+                                      const void* r, void* y, int bf16, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_TESTING_H_ */

@@ -1,0 +1,177 @@
+"""Python binding of libwkv.so, the B200 (sm_100a) WKV library.
+
+Argument marshalling only: every function checks the torch tensors it is given (device,
+dtype, contiguity, shape), allocates outputs the caller did not pass, and calls the C
+entry point of the same name (include/wkv.h) on the current CUDA stream. All arithmetic
+runs in the library's CUDA kernels; there is no fallback. Importing this package fails
+loudly when libwkv.so has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
+           "wkv_stream_status", "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m rwkv_linear_attention_wkv_b200.build`"
+        " (the WKV operator has no non-CUDA implementation)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int64
+_SIGS = {
+    "wkv_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "wkv_version": ([], ctypes.c_int),
+    "wkv_forward": ([_I, _I, _I] + [_P] * 6 + [_P], ctypes.c_int),
+    "wkv_forward_bf16": ([_I, _I, _I] + [_P] * 6 + [_P], ctypes.c_int),
+    "wkv_forward_state": ([_I, _I, _I] + [_P] * 12 + [_P], ctypes.c_int),
+    "wkv_decode_step": ([_I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
+    "wkv_stream_status": ([_P], ctypes.c_int),
+    "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
+    "wkv_testing_forward_plain": ([_I, _I, _I] + [_P] * 6 + [ctypes.c_int, _P], ctypes.c_int),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+class WkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {wkv_status_string(status)} ({status})")
+        self.status = status
+
+
+def wkv_status_string(status: int) -> str:
+    return lib.wkv_status_string(int(status)).decode()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t, name, dtype, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _call(fn, *args):
+    rc = getattr(lib, fn)(*args)
+    if rc != 0:
+        raise WkvError(fn, rc)
+
+
+def _fwd_common(w, u, k, v, r, y, dtype):
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    _need(k, "k", dtype)
+    _need(v, "v", dtype, (B, T, C))
+    if r is not None:
+        _need(r, "r", dtype, (B, T, C))
+    _need(w, "w", torch.float32, (C,))
+    _need(u, "u", torch.float32, (C,))
+    if y is None:
+        y = torch.empty((B, T, C), dtype=dtype, device=k.device)
+    _need(y, "y", dtype, (B, T, C))
+    return B, T, C, y
+
+
+def wkv_forward(w, u, k, v, r=None, y=None, stream=None):
+    """fp32 forward: y = sigmoid(r) * wkv (no gate when r is None). Returns y."""
+    torch = _torch()
+    B, T, C, y = _fwd_common(w, u, k, v, r, y, torch.float32)
+    _call("wkv_forward", B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
+          _stream(stream))
+    return y
+
+
+def wkv_forward_bf16(w, u, k, v, r=None, y=None, stream=None):
+    """bf16 in/out forward (fp32 arithmetic). Returns y (bf16)."""
+    torch = _torch()
+    B, T, C, y = _fwd_common(w, u, k, v, r, y, torch.bfloat16)
+    _call("wkv_forward_bf16", B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
+          _stream(stream))
+    return y
+
+
+def wkv_forward_state(w, u, k, v, r=None, state=None, y=None, state_out=None,
+                      want_state=True, stream=None):
+    """fp32 forward with state. state = (a, b, p) fp32 [B, C] or None (empty).
+
+    Returns (y, (a1, b1, p1)), or (y, None) with want_state=False. state_out may be given
+    (and may be the same tensors as state) to write the final state in place.
+    """
+    torch = _torch()
+    B, T, C, y = _fwd_common(w, u, k, v, r, y, torch.float32)
+    a0 = b0 = p0 = None
+    if state is not None:
+        a0, b0, p0 = state
+        for n, t in (("a0", a0), ("b0", b0), ("p0", p0)):
+            _need(t, n, torch.float32, (B, C))
+    a1 = b1 = p1 = None
+    if want_state:
+        if state_out is None:
+            state_out = tuple(torch.empty((B, C), dtype=torch.float32, device=k.device)
+                              for _ in range(3))
+        a1, b1, p1 = state_out
+        for n, t in (("a1", a1), ("b1", b1), ("p1", p1)):
+            _need(t, n, torch.float32, (B, C))
+    _call("wkv_forward_state", B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
+          _ptr(a0), _ptr(b0), _ptr(p0), _ptr(a1), _ptr(b1), _ptr(p1), _stream(stream))
+    return y, ((a1, b1, p1) if want_state else None)
+
+
+def wkv_decode_step(w, u, k, v, r, a, b, p, y=None, stream=None):
+    """One token for [N, L, C] states; w, u [L, C]; (a, b, p) updated in place. Returns y."""
+    torch = _torch()
+    if k.dim() != 3:
+        raise ValueError("k must be (N, L, C)")
+    N, L, C = k.shape
+    f32 = torch.float32
+    _need(k, "k", f32)
+    for n, t in (("v", v), ("a", a), ("b", b), ("p", p)):
+        _need(t, n, f32, (N, L, C))
+    if r is not None:
+        _need(r, "r", f32, (N, L, C))
+    _need(w, "w", f32, (L, C))
+    _need(u, "u", f32, (L, C))
+    if y is None:
+        y = torch.empty((N, L, C), dtype=f32, device=k.device)
+    _need(y, "y", f32, (N, L, C))
+    _call("wkv_decode_step", N, L, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
+          _ptr(a), _ptr(b), _ptr(p), _stream(stream))
+    return y
+
+
+def wkv_stream_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device-side status code."""
+    return int(lib.wkv_stream_status(_stream(stream)))

@@ -1,0 +1,256 @@
+// WKV forward over full sequences, one thread per (b, c) channel (sm_100a).
+//
+// Streaming kernel: one warp per CTA owns 32 adjacent channels of one batch row and walks
+// the whole sequence. Tiles of [TT tokens x 32 channels] of k, v, r are brought into
+// shared memory by TMA (3-D tensor maps over (C, T, B), so ragged T and C edges are
+// zero-filled on load and clipped on store), S stages deep, each stage on its own
+// mbarrier. y is staged in shared memory and written back by TMA store. The channel
+// state (a, b, P) lives in registers for the whole sequence.
+//
+// A plain kernel (direct coalesced global loads, same arithmetic) serves shapes the TMA
+// path cannot describe: C not a multiple of 4 (fp32) / 8 (bf16), or base pointers that
+// are not 16-byte aligned.
+#include <cuda.h>
+
+#include "wkv_internal.h"
+#include "wkv_step.cuh"
+
+namespace wkv {
+
+// Process n tokens of a tile already in shared memory (rows of 32 elements, this lane's
+// column), in windows of RB tokens. FULL: n == TT, fully unrolled.
+template <typename Tin, bool GATE, bool FASTOUT, int TT, int RB, bool FULL>
+__device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, const Tin* K,
+                                            const Tin* V, const Tin* R, Tin* Y, int n) {
+  if (FULL) {
+#pragma unroll
+    for (int w0 = 0; w0 < TT; w0 += RB) {
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        const int row = (w0 + j) * 32;
+        const float k = Elem<Tin>::to_f(K[row]);
+        const float v = Elem<Tin>::to_f(V[row]);
+        const float r = GATE ? Elem<Tin>::to_f(R[row]) : 0.f;
+        Y[row] = Elem<Tin>::from_f(wkv_token<GATE, FASTOUT>(s, cp, float(j + 1), k, v, r));
+      }
+      wkv_rebase(s, float(RB) * cp.w2);
+    }
+  } else {
+    int j = 0;
+    for (int t = 0; t < n; ++t) {
+      const int row = t * 32;
+      const float k = Elem<Tin>::to_f(K[row]);
+      const float v = Elem<Tin>::to_f(V[row]);
+      const float r = GATE ? Elem<Tin>::to_f(R[row]) : 0.f;
+      Y[row] = Elem<Tin>::from_f(wkv_token<GATE, FASTOUT>(s, cp, float(j + 1), k, v, r));
+      if (++j == RB) {
+        wkv_rebase(s, float(RB) * cp.w2);
+        j = 0;
+      }
+    }
+    if (j) wkv_rebase(s, float(j) * cp.w2);
+  }
+}
+
+template <typename Tin, bool GATE, int TT, int S, int RB>
+__global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_y, int T,
+    int C, const float* __restrict__ w, const float* __restrict__ u, const float* a0,
+    const float* b0, const float* p0, float* a1, float* b1, float* p1, unsigned* err) {
+  constexpr int kTile = TT * 32;
+  constexpr uint32_t kTileBytes = kTile * sizeof(Tin);
+  constexpr uint32_t kStageBytes = (GATE ? 3u : 2u) * kTileBytes;
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Tin* sk = reinterpret_cast<Tin*>(smem_raw);
+  Tin* sv = sk + S * kTile;
+  Tin* sr = sv + S * kTile;                      // unused without the gate
+  Tin* sy = sr + (GATE ? S * kTile : 0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sy + S * kTile);
+
+  const int lane = threadIdx.x;
+  const int G = (C + 31) >> 5;
+  const int b = blockIdx.x / G;
+  const int g = blockIdx.x - b * G;
+  const int c = (g << 5) + lane;
+  const bool valid = c < C;
+  const int ntiles = (T + TT - 1) / TT;
+
+  auto issue = [&](int stage, int tile) {
+    uint64_t* bar = &bars[stage];
+    mbar_arrive_expect_tx(bar, kStageBytes);
+    tma_load_3d(sk + stage * kTile, &tm_k, bar, g << 5, tile * TT, b);
+    tma_load_3d(sv + stage * kTile, &tm_v, bar, g << 5, tile * TT, b);
+    if (GATE) tma_load_3d(sr + stage * kTile, &tm_r, bar, g << 5, tile * TT, b);
+  };
+
+  if (lane == 0) {
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    if (GATE) prefetch_tmap(&tm_r);
+    prefetch_tmap(&tm_y);
+#pragma unroll
+    for (int st = 0; st < S; ++st) mbar_init(&bars[st], 1);
+    mbar_fence_init();
+    for (int st = 0; st < S && st < ntiles; ++st) issue(st, st);
+  }
+  __syncwarp();
+
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
+  const size_t sidx = size_t(b) * C + c;
+  const bool has_state = a0 != nullptr;
+  ChanState s = (has_state && valid) ? load_state(a0[sidx], b0[sidx], p0[sidx]) : empty_state();
+  const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int st = i % S;
+    mbar_wait(&bars[st], (i / S) & 1, err);
+    if (lane == 0 && i >= S) tma_store_wait_read<S - 1>();
+    __syncwarp();
+    const Tin* K = sk + st * kTile + lane;
+    const Tin* V = sv + st * kTile + lane;
+    const Tin* R = sr + st * kTile + lane;
+    Tin* Y = sy + st * kTile + lane;
+    const int n = min(TT, T - i * TT);
+    if (n == TT) {
+      if (fast)
+        tile_tokens<Tin, GATE, true, TT, RB, true>(s, cp, K, V, R, Y, n);
+      else
+        tile_tokens<Tin, GATE, false, TT, RB, true>(s, cp, K, V, R, Y, n);
+    } else {
+      if (fast)
+        tile_tokens<Tin, GATE, true, TT, RB, false>(s, cp, K, V, R, Y, n);
+      else
+        tile_tokens<Tin, GATE, false, TT, RB, false>(s, cp, K, V, R, Y, n);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(&tm_y, sy + st * kTile, g << 5, i * TT, b);
+      tma_store_commit();
+      if (i + S < ntiles) issue(st, i + S);
+    }
+  }
+  if (lane == 0) tma_store_wait_all();
+
+  if (a1 != nullptr && valid) {
+    a1[sidx] = s.a;
+    b1[sidx] = s.b;
+    p1[sidx] = (T == 0 && has_state) ? p0[sidx] : state_log_scale(s);
+  }
+}
+
+// Plain kernel: one thread per (b, c), coalesced across threads, no shared memory.
+template <typename Tin, bool GATE, int RB>
+__global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
+    int64_t B, int64_t T, int64_t C, const float* __restrict__ w, const float* __restrict__ u,
+    const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ r,
+    Tin* __restrict__ y, const float* a0, const float* b0, const float* p0, float* a1, float* b1,
+    float* p1) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const bool valid = idx < B * C;
+  const int64_t bb = valid ? idx / C : 0;
+  const int64_t c = valid ? idx - bb * C : 0;
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
+  const bool has_state = a0 != nullptr;
+  ChanState s = (has_state && valid) ? load_state(a0[idx], b0[idx], p0[idx]) : empty_state();
+  const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+  if (!valid) return;
+  const int64_t base = bb * T * C + c;
+  int j = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t e = base + t * C;
+    const float kk = Elem<Tin>::to_f(k[e]);
+    const float vv = Elem<Tin>::to_f(v[e]);
+    const float rr = GATE ? Elem<Tin>::to_f(r[e]) : 0.f;
+    const float out = fast ? wkv_token<GATE, true>(s, cp, float(j + 1), kk, vv, rr)
+                           : wkv_token<GATE, false>(s, cp, float(j + 1), kk, vv, rr);
+    y[e] = Elem<Tin>::from_f(out);
+    if (++j == RB) {
+      wkv_rebase(s, float(RB) * cp.w2);
+      j = 0;
+    }
+  }
+  if (j) wkv_rebase(s, float(j) * cp.w2);
+  if (a1 != nullptr) {
+    a1[idx] = s.a;
+    b1[idx] = s.b;
+    p1[idx] = (T == 0 && has_state) ? p0[idx] : state_log_scale(s);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr int kTT = 32;   // tokens per tile
+constexpr int kRB = 16;   // tokens per log-scale window
+
+template <typename Tin>
+constexpr int stages() {
+  return 3;
+}
+
+template <typename Tin, bool GATE>
+size_t tma_smem_bytes() {
+  return size_t(stages<Tin>()) * (GATE ? 4 : 3) * kTT * 32 * sizeof(Tin) +
+         stages<Tin>() * sizeof(uint64_t);
+}
+
+template <typename Tin, bool GATE>
+int launch_tma(const FwdArgs& a, cudaStream_t stream) {
+  CUtensorMap tk, tv, tr, ty;
+  const CUtensorMapDataType dt =
+      sizeof(Tin) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  int rc = encode_btc_map(&tk, a.k, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
+  if (!rc) rc = encode_btc_map(&tv, a.v, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
+  if (!rc) rc = encode_btc_map(&tr, GATE ? a.r : a.k, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
+  if (!rc) rc = encode_btc_map(&ty, a.y, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
+  if (rc) return rc;
+  auto kern = wkv_fwd_tma_kernel<Tin, GATE, kTT, stages<Tin>(), kRB>;
+  const size_t smem = tma_smem_bytes<Tin, GATE>();
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return WKV_ERR_CUDA;
+  const int64_t G = (a.C + 31) / 32;
+  const int64_t grid = a.B * G;
+  kern<<<unsigned(grid), 32, smem, stream>>>(tk, tv, tr, ty, int(a.T), int(a.C), a.w, a.u, a.a0,
+                                             a.b0, a.p0, a.a1, a.b1, a.p1, a.err);
+  return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename Tin, bool GATE>
+int launch_plain(const FwdArgs& a, cudaStream_t stream) {
+  const int64_t n = a.B * a.C;
+  const int block = 128;
+  const int64_t grid = (n + block - 1) / block;
+  wkv_fwd_plain_kernel<Tin, GATE, kRB><<<unsigned(grid), block, 0, stream>>>(
+      a.B, a.T, a.C, a.w, a.u, static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
+      static_cast<const Tin*>(a.r), static_cast<Tin*>(a.y), a.a0, a.b0, a.p0, a.a1, a.b1, a.p1);
+  return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <typename Tin>
+int dispatch(const FwdArgs& a, bool use_tma, cudaStream_t stream) {
+  const bool gate = a.r != nullptr;
+  if (use_tma) return gate ? launch_tma<Tin, true>(a, stream) : launch_tma<Tin, false>(a, stream);
+  return gate ? launch_plain<Tin, true>(a, stream) : launch_plain<Tin, false>(a, stream);
+}
+
+}  // namespace
+
+bool fwd_tma_ok(const FwdArgs& a, int elem_bytes) {
+  auto al16 = [](const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  return (a.C * elem_bytes) % 16 == 0 && al16(a.k) && al16(a.v) && al16(a.r) && al16(a.y) &&
+         a.T < (int64_t(1) << 31) && a.C < (int64_t(1) << 31) && a.B < (int64_t(1) << 31) &&
+         a.B * ((a.C + 31) / 32) < (int64_t(1) << 31);
+}
+
+int launch_fwd_stream(const FwdArgs& a, bool bf16, bool force_plain, cudaStream_t stream) {
+  const bool tma = !force_plain && fwd_tma_ok(a, bf16 ? 2 : 4);
+  return bf16 ? dispatch<__nv_bfloat16>(a, tma, stream) : dispatch<float>(a, tma, stream);
+}
+
+}  // namespace wkv

@@ -1,0 +1,71 @@
+// Internal interfaces between the C-ABI layer (wkv_api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "wkv.h"
+
+namespace wkv {
+
+// Arguments of one forward pass over (B, T, C). k, v, r, y are fp32 or bf16 according to
+// the entry point; r may be null (no gate); a0/b0/p0 null = empty initial state; a1/b1/p1
+// null = final state not wanted.
+struct FwdArgs {
+  int64_t B, T, C;
+  const float* w;
+  const float* u;
+  const void* k;
+  const void* v;
+  const void* r;
+  void* y;
+  const float* a0;
+  const float* b0;
+  const float* p0;
+  float* a1;
+  float* b1;
+  float* p1;
+  unsigned* err;  // device error word
+};
+
+// 3-D tiled tensor map over a (B, T, C) tensor (C fastest) with a box of
+// [box_c channels x box_t tokens x 1 batch row]. Returns a wkv_status.
+int encode_btc_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                   int elem_bytes, int64_t B, int64_t T, int64_t C, int box_c, int box_t);
+
+// Whether the TMA streaming kernel can describe this problem (alignment, extents).
+bool fwd_tma_ok(const FwdArgs& a, int elem_bytes);
+
+// Whole-sequence forward, one thread per channel (streaming TMA kernel, or the plain
+// kernel when the TMA kernel cannot be used or force_plain is set).
+int launch_fwd_stream(const FwdArgs& a, bool bf16, bool force_plain, cudaStream_t stream);
+
+// Chunked (time-parallel) forward for problems with few channels; fp32 only.
+// scratch: device memory of chunked_scratch_bytes(); its first flag_bytes must be
+// zero on entry (the caller clears them).
+size_t chunked_scratch_bytes(int64_t B, int64_t T, int64_t C, int64_t* flag_bytes,
+                             int* n_segments);
+int launch_fwd_chunked(const FwdArgs& a, void* scratch, int n_segments, cudaStream_t stream);
+// Same, with the look-back wait limit (ns) given and, for tests of the bounded wait,
+// segment 0 optionally withholding its inclusive prefix so that its successors give up.
+int launch_fwd_chunked_ex(const FwdArgs& a, void* scratch, int n_segments,
+                          unsigned long long wait_ns, int withhold_seg0, cudaStream_t stream);
+
+// One decode step over N x L x C states.
+struct DecodeArgs {
+  int64_t N, L, C;
+  const float* w;
+  const float* u;
+  const float* k;
+  const float* v;
+  const float* r;
+  float* y;
+  float* a;
+  float* b;
+  float* p;
+};
+int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+}  // namespace wkv

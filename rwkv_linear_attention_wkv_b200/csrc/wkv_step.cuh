@@ -1,0 +1,141 @@
+// The per-channel WKV recurrence in log-max-stabilised, base-2 form (sm_100a).
+//
+// Definition (concept page "RWKV（Receptance Weighted Key Value）概念", section 3.2, and the
+// paper notes "RWKV - 把 RNN 重新带回 Transformer 时代的线性大模型", "一句话总结"):
+//   wkv_t = (A_{t-1} + e^{u+k_t} v_t) / (B_{t-1} + e^{u+k_t}),   y_t = sigmoid(r_t) wkv_t
+//   A_t = e^{-w} A_{t-1} + e^{k_t} v_t,   B_t = e^{-w} B_{t-1} + e^{k_t}.
+// The notes name a stabilising exponent p in the inference state but give no formula; the
+// reading used here is A = a 2^P, B = b 2^P with P the running maximum of the (decayed)
+// log2-weights, so that one of the two factors of every update is exactly 1.
+//
+// Representation per channel: (a, b) scaled numerator and denominator, and the log2-scale
+// P_t kept as an exact pair of floats across "windows" of consecutive tokens:
+//   * at the start of a window, P = Q + pl with Q, pl floats (|pl| <= ulp(Q)/2);
+//   * token j = 1..n of the window has the log2-weight m_j = k_j log2(e) + j w2 - pl,
+//     measured against the window start (w2 = w log2(e)); Q tracks max(Q, m_j);
+//   * at the end of the window P = Q + pl - n w2 is re-split exactly (TwoSum).
+// Decaying the scale by w2 once per token in float would round the same way every step
+// (the low bits of w2 below ulp(P) are constant) and drift by up to ulp(P)/2 per token;
+// the window form rounds each m_j once and never accumulates.
+//
+// Per token (d = m_j - Q; one of e1, e2 is 1, the other 2^{-|d|}):
+//   state update   a' = e1 a + e2 v,  b' = e1 b + e2,  Q' = max(Q, m_j)
+//   output         with H = 2^{u2 - w2} = e^{u-w}:
+//                  wkv = (e1 a + H e2 v) / (e1 b + H e2)
+// i.e. numerator and denominator of the output scaled by e^{-w} 2^{-P_t}, which is the
+// scale of the updated state, so the output costs no exponential of its own. This needs
+// H to be a normal float; for |u - w| beyond ~69 (nats) the generic form below takes
+// over, which stabilises the output with its own exponential.
+#pragma once
+
+#include "wkv_device.cuh"
+
+namespace wkv {
+
+struct ChanState {
+  float a, b;   // scaled numerator / denominator
+  float Q, pl;  // log2-scale of the state: Q + pl (see above)
+};
+
+struct ChanParams {
+  float w2;   // w log2(e)
+  float uw2;  // (u - w) log2(e)
+  float H;    // 2^{uw2}
+};
+
+// |u - w| log2(e) bound for the single-exponential output form.
+constexpr float kFastOutBound = 100.0f;
+
+__device__ __forceinline__ ChanParams chan_params(float w, float u) {
+  ChanParams p;
+  p.w2 = w * kLog2e;
+  p.uw2 = fmaf(u, kLog2e, -p.w2);
+  p.H = ex2(p.uw2);
+  return p;
+}
+
+__device__ __forceinline__ ChanState empty_state() {
+  ChanState s;
+  s.a = 0.f;
+  s.b = 0.f;
+  s.Q = kEmptyLogScale;
+  s.pl = 0.f;
+  return s;
+}
+
+// State given as (a, b, p) with A = a e^p, B = b e^p (p in natural log).
+__device__ __forceinline__ ChanState load_state(float a, float b, float p) {
+  ChanState s;
+  s.a = a;
+  s.b = b;
+  s.Q = p * kLog2e;
+  s.pl = fmaf(p, kLog2e, -s.Q);  // exact low part of the product
+  return s;
+}
+
+// Natural-log scale of the state (one rounding).
+__device__ __forceinline__ float state_log_scale(const ChanState& s) {
+  return fmaf(s.Q, kLn2, s.pl * kLn2);
+}
+
+// One token; fj = j as float (1-based position within the window).
+template <bool GATE, bool FASTOUT>
+__device__ __forceinline__ float wkv_token(ChanState& s, const ChanParams& cp, float fj, float k,
+                                           float v, float r) {
+  const float m = fmaf(fj, cp.w2, fmaf(k, kLog2e, -s.pl));
+  const float d = m - s.Q;
+  const float e = ex2(-fabsf(d));
+  const bool c = d > 0.f;
+  const float e1 = c ? e : 1.f;
+  const float e2 = c ? 1.f : e;
+  s.Q = fmaxf(s.Q, m);
+  float num, den;
+  if (FASTOUT) {
+    const float he = cp.H * e2;
+    num = fmaf(e1, s.a, he * v);
+    den = fmaf(e1, s.b, he);
+  } else {
+    // Output stabilised on its own: exponent of the current token against the state
+    // before it is d + (u - w) log2(e).
+    const float dO = d + cp.uw2;
+    const float o = ex2(-fabsf(dO));
+    const bool co = dO > 0.f;
+    const float o1 = co ? o : 1.f;
+    const float o2 = co ? 1.f : o;
+    num = fmaf(o1, s.a, o2 * v);
+    den = fmaf(o1, s.b, o2);
+  }
+  if (GATE) {
+    // sigmoid(r) folded into the division: y = num / (den (1 + e^{-r})).
+    const float er = ex2(r * -kLog2e);
+    den = fmaf(den, er, den);
+  }
+  s.a = fmaf(e1, s.a, e2 * v);
+  s.b = fmaf(e1, s.b, e2);
+  return num * rcp(den);
+}
+
+// State update only (no output): used for chunk aggregates and recomputation.
+__device__ __forceinline__ void wkv_absorb(ChanState& s, const ChanParams& cp, float fj, float k,
+                                           float v) {
+  const float m = fmaf(fj, cp.w2, fmaf(k, kLog2e, -s.pl));
+  const float d = m - s.Q;
+  const float e = ex2(-fabsf(d));
+  const bool c = d > 0.f;
+  const float e1 = c ? e : 1.f;
+  const float e2 = c ? 1.f : e;
+  s.Q = fmaxf(s.Q, m);
+  s.a = fmaf(e1, s.a, e2 * v);
+  s.b = fmaf(e1, s.b, e2);
+}
+
+// End of a window of n tokens: P = Q + pl - n w2, re-split exactly.
+__device__ __forceinline__ void wkv_rebase(ChanState& s, float nw2) {
+  const float c2 = s.pl - nw2;
+  float hi, lo;
+  two_sum(s.Q, c2, hi, lo);
+  s.Q = hi;
+  s.pl = lo;
+}
+
+}  // namespace wkv

@@ -1,0 +1,227 @@
+"""GPU parity of the forward entry points against the fp64 oracle (through the C ABI).
+
+Every case runs the library's CUDA kernels on seeded inputs from wkv_inputs and compares
+elementwise with the oracle on the same stored values (bf16 inputs upcast exactly).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import wkv_inputs
+from wkv_check import assert_bf16_close, assert_fp32_close, assert_state_close
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def W():
+    import rwkv_linear_attention_wkv_b200 as W
+    return W
+
+
+def dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host_bf16(t):
+    return wkv_inputs.bf16_bits_to_f32(t.view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def run_f32(W, x, gate=True, plain=False, T_slice=None):
+    w, u, k, v, r = dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(x.r) if gate else None
+    if plain:
+        import ctypes
+        y = torch.empty_like(k)
+        rc = W.lib.wkv_testing_forward_plain(x.B, x.T, x.C, ctypes.c_void_p(w.data_ptr()),
+                                             ctypes.c_void_p(u.data_ptr()),
+                                             ctypes.c_void_p(k.data_ptr()),
+                                             ctypes.c_void_p(v.data_ptr()),
+                                             ctypes.c_void_p(r.data_ptr()) if gate else None,
+                                             ctypes.c_void_p(y.data_ptr()), 0,
+                                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert rc == 0, W.wkv_status_string(rc)
+    else:
+        y = W.wkv_forward(w, u, k, v, r)
+    assert W.wkv_stream_status() == 0
+    return y.cpu().numpy()
+
+
+def test_tiny_forward_matches_parallel_form(W):
+    x = wkv_inputs.tiny_forward(seed=0)
+    y = run_f32(W, x)
+    ref = oracle.wkv_direct(x.w, x.u, x.k, x.v, x.r)
+    assert_fp32_close(y, ref)
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 4), (2, 1, 64), (1, 33, 32), (3, 100, 96),
+                                   (2, 257, 40), (1, 64, 37), (2, 31, 5), (1, 5, 1)])
+@pytest.mark.parametrize("gate", [True, False])
+def test_ragged_shapes_fp32(W, shape, gate):
+    B, T, C = shape
+    x = wkv_inputs.make_inputs(B, T, C, seed=B * 1000 + T * 10 + C, k_std=2.0)
+    ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r if gate else None)
+    assert_fp32_close(run_f32(W, x, gate), ref)
+    assert_fp32_close(run_f32(W, x, gate, plain=True), ref, "y (plain kernel)")
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 8), (2, 77, 64), (1, 300, 200), (3, 40, 13)])
+def test_ragged_shapes_bf16(W, shape):
+    B, T, C = shape
+    x = wkv_inputs.make_inputs(B, T, C, seed=7 + T, dtype="bf16", logw_range=(-6, 2),
+                               u_bound=2.0, k_std=3.0, spike_frac=0.01)
+    y = W.wkv_forward_bf16(dev(x.w), dev(x.u), dev_bf16(x.bits["k"]), dev_bf16(x.bits["v"]),
+                           dev_bf16(x.bits["r"]))
+    assert W.wkv_stream_status() == 0
+    ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r)
+    assert_bf16_close(host_bf16(y), ref)
+
+
+def test_single_token_is_v_and_constant_v(W):
+    x = wkv_inputs.make_inputs(3, 1, 64, seed=3, k_std=5.0)
+    y = run_f32(W, x, gate=False)
+    np.testing.assert_allclose(y, x.v, rtol=5e-7, atol=0)
+    x = wkv_inputs.make_inputs(2, 200, 64, seed=4, k_std=3.0)
+    x.v[:] = np.linspace(-3, 3, 64, dtype=np.float32)
+    y = run_f32(W, x, gate=False)
+    assert_fp32_close(y, np.broadcast_to(x.v, y.shape), tol=1e-6)
+
+
+def test_extreme_parameters_use_generic_output(W):
+    # |u - w| large: the single-exponential output scale 2^{(u-w) log2 e} would leave the
+    # float range; the kernel switches to the separately stabilised output.
+    x = wkv_inputs.make_inputs(2, 70, 64, seed=5, k_std=2.0)
+    x.w[:32] = 90.0
+    x.u[32:] = 95.0
+    ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r)
+    assert_fp32_close(run_f32(W, x), ref)
+    assert_fp32_close(run_f32(W, x, plain=True), ref)
+
+
+def test_empty_problems(W):
+    z = torch.empty((0,), device="cuda")
+    w = torch.ones(8, device="cuda")
+    for B, T, C in ((0, 5, 8), (2, 0, 8), (2, 5, 0)):
+        k = torch.zeros((B, T, C), device="cuda")
+        W.wkv_forward(torch.ones(C, device="cuda"), torch.zeros(C, device="cuda"), k, k, k)
+    assert W.wkv_stream_status() == 0
+    # T = 0 with state: the final state is the initial state.
+    a0 = torch.randn(2, 8, device="cuda")
+    b0 = torch.rand(2, 8, device="cuda") + 0.5
+    p0 = torch.randn(2, 8, device="cuda")
+    k = torch.zeros((2, 0, 8), device="cuda")
+    _, (a1, b1, p1) = W.wkv_forward_state(w, w, k, k, k, state=(a0, b0, p0))
+    assert torch.equal(a1, a0) and torch.equal(b1, b0) and torch.equal(p1, p0)
+    del z
+
+
+def test_invalid_arguments_raise(W):
+    k = torch.zeros((1, 4, 8), device="cuda")
+    with pytest.raises(ValueError):
+        W.wkv_forward(torch.ones(7, device="cuda"), torch.zeros(8, device="cuda"), k, k)
+    with pytest.raises(TypeError):
+        W.wkv_forward(torch.ones(8, device="cuda"), torch.zeros(8, device="cuda"),
+                      k.double(), k.double())
+
+
+def test_training_shape_forward(W):
+    # B*C = 12288 channels: the chunked (time-parallel) kernel.
+    x = wkv_inputs.training_shape(seed=0)
+    ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r)
+    assert_fp32_close(run_f32(W, x), ref, "y (chunked)")
+    assert_fp32_close(run_f32(W, x, plain=True), ref, "y (plain)")
+    for b, c in wkv_inputs.sample_channels(x.B, x.C, 4):
+        yd = oracle.wkv_direct(x.w[c:c + 1], x.u[c:c + 1], x.k[b:b + 1, :, c:c + 1],
+                               x.v[b:b + 1, :, c:c + 1], x.r[b:b + 1, :, c:c + 1])
+        np.testing.assert_allclose(yd[0, :, 0], ref[b, :, c], rtol=1e-11, atol=1e-12)
+
+
+def test_long_bf16_full_size(W):
+    # The 7B-shaped bf16 workload, B=8, T=4096, C=4096, k spikes of +60; every element.
+    x = wkv_inputs.long_bf16(seed=0)
+    y = W.wkv_forward_bf16(dev(x.w), dev(x.u), dev_bf16(x.bits["k"]), dev_bf16(x.bits["v"]),
+                           dev_bf16(x.bits["r"]))
+    assert W.wkv_stream_status() == 0
+    yh = host_bf16(y)
+    del y
+    stats = {"strict_1ulp_violations": 0, "n": 0, "max_err_in_ulps": 0.0}
+    for b in range(x.B):          # one batch row at a time bounds host memory
+        ref = oracle.wkv_recurrent(x.w, x.u, x.k[b:b + 1], x.v[b:b + 1], x.r[b:b + 1])
+        s = assert_bf16_close(yh[b:b + 1], ref, f"y[b={b}]")
+        stats["strict_1ulp_violations"] += s["strict_1ulp_violations"]
+        stats["n"] += s["n"]
+        stats["max_err_in_ulps"] = max(stats["max_err_in_ulps"], s["max_err_in_ulps"])
+    print("bf16 full-size parity:", stats)
+    for b, c in wkv_inputs.sample_channels(x.B, x.C, 3):
+        yd = oracle.wkv_direct(x.w[c:c + 1], x.u[c:c + 1], x.k[b:b + 1, :, c:c + 1],
+                               x.v[b:b + 1, :, c:c + 1], x.r[b:b + 1, :, c:c + 1])
+        assert_bf16_close(yh[b, :, c], yd[0, :, 0], f"y[{b},:,{c}] vs parallel form")
+
+
+def test_long_context_full_size_with_state(W):
+    # One sequence of 32768 tokens x 4096 channels: the chunked kernel; final state too.
+    x = wkv_inputs.long_context(seed=0)
+    w, u, k, v, r = dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(x.r)
+    y, (a1, b1, p1) = W.wkv_forward_state(w, u, k, v, r)
+    assert W.wkv_stream_status() == 0
+    ref, A, Bd = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r, want_state=True)
+    assert_fp32_close(y.cpu().numpy(), ref)
+    assert_state_close(a1.cpu().numpy(), b1.cpu().numpy(), p1.cpu().numpy(), A, Bd)
+
+
+def test_long_context_stress_distributions(W):
+    # Same shape with k ~ N(0,3) and +60 spikes, w up to e^2 (shorter, to bound time).
+    x = wkv_inputs.long_context(seed=1, T=8192, C=2048, stress=True)
+    y, (a1, b1, p1) = W.wkv_forward_state(dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(x.r))
+    assert W.wkv_stream_status() == 0
+    ref, A, Bd = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r, want_state=True)
+    assert_fp32_close(y.cpu().numpy(), ref)
+    assert_state_close(a1.cpu().numpy(), b1.cpu().numpy(), p1.cpu().numpy(), A, Bd)
+
+
+@pytest.mark.parametrize("B,T,C,split", [(2, 700, 64, 333), (1, 3000, 128, 1024),
+                                         (40, 100, 512, 37)])
+def test_split_invariance(W, B, T, C, split):
+    x = wkv_inputs.make_inputs(B, T, C, seed=T + split, k_std=2.0)
+    w, u, k, v, r = dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(x.r)
+    y, st = W.wkv_forward_state(w, u, k, v, r)
+    y1, st1 = W.wkv_forward_state(w, u, k[:, :split].contiguous(), v[:, :split].contiguous(),
+                                  r[:, :split].contiguous())
+    y2, st2 = W.wkv_forward_state(w, u, k[:, split:].contiguous(), v[:, split:].contiguous(),
+                                  r[:, split:].contiguous(), state=st1, state_out=st1)
+    assert W.wkv_stream_status() == 0
+    ref, A, Bd = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r, want_state=True)
+    assert_fp32_close(torch.cat([y1, y2], 1).cpu().numpy(), ref)
+    assert_fp32_close(y.cpu().numpy(), ref)
+    for s in (st, st2):
+        assert_state_close(*(t.cpu().numpy() for t in s), A, Bd)
+
+
+def test_initial_state_matches_oracle(W):
+    x = wkv_inputs.make_inputs(3, 500, 96, seed=11, k_std=2.0)
+    g = np.random.Generator(np.random.PCG64(5))
+    a0 = g.standard_normal((3, 96)).astype(np.float32)
+    b0 = g.uniform(0.5, 2, (3, 96)).astype(np.float32)
+    p0 = g.standard_normal((3, 96)).astype(np.float32)
+    A0, B0 = oracle.state_from_scaled(a0, b0, p0)
+    ref, A, Bd = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r, A0, B0, want_state=True)
+    y, st = W.wkv_forward_state(dev(x.w), dev(x.u), dev(x.k), dev(x.v), dev(x.r),
+                                state=(dev(a0), dev(b0), dev(p0)))
+    assert W.wkv_stream_status() == 0
+    assert_fp32_close(y.cpu().numpy(), ref)
+    assert_state_close(*(t.cpu().numpy() for t in st), A, Bd)
+
+
+def test_lookback_wait_gives_up_and_reports(W):
+    import ctypes
+    s = torch.cuda.current_stream()
+    rc = W.lib.wkv_testing_lookback_timeout(1_000_000, ctypes.c_void_p(s.cuda_stream))
+    assert rc == 0
+    assert W.wkv_stream_status() == 4          # WKV_ERR_TIMEOUT
+    assert W.wkv_stream_status() == 0          # cleared
+    x = wkv_inputs.tiny_forward(seed=0)        # context still usable
+    assert_fp32_close(run_f32(W, x), oracle.wkv_direct(x.w, x.u, x.k, x.v, x.r))

@@ -13,8 +13,10 @@ Recipe (all draws from ``numpy.random.Generator(PCG64(seed))``, in this order):
 * optionally a Bernoulli(spike_frac) mask over (B, T, C) whose entries of k are set
   to ``spike_value`` (overflow stress).
 
-Values are drawn in float64 and rounded to float32 (round to nearest even); for bf16
-storage the float32 values are rounded once more to bf16 (round to nearest even).
+The per-channel parameters are drawn in float64 and rounded to float32. The (B, T, C)
+tensors are drawn as float32 standard normals (NumPy's float32 ziggurat, about five
+times faster than float64 draws, which matters at 10^8 elements) and scaled by k_std in
+float32; for bf16 storage the float32 values are rounded to bf16 (round to nearest even).
 The arrays handed out are the *stored* values: float32 arrays, or, for bf16, the
 float32 arrays holding exactly the bf16 values plus the raw uint16 bit patterns.
 """
@@ -28,8 +30,12 @@ import numpy as np
 def round_to_bf16_bits(x32: np.ndarray) -> np.ndarray:
     """float32 -> bf16 bit patterns (uint16), round to nearest even. NaN-free input."""
     u = np.ascontiguousarray(x32, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    return ((u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+    r = u >> np.uint32(16)
+    r &= np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r >>= np.uint32(16)
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -54,8 +60,7 @@ class WkvInputs:
     bits: dict = field(default_factory=dict)  # bf16 only: name -> uint16 [B, T, C]
 
 
-def _store(x64: np.ndarray, dtype: str):
-    x32 = x64.astype(np.float32)
+def _store(x32: np.ndarray, dtype: str):
     if dtype == "f32":
         return x32, None
     if dtype == "bf16":
@@ -74,17 +79,20 @@ def make_inputs(B: int, T: int, C: int, seed: int = 0, *, dtype: str = "f32",
     w = np.exp(logw).astype(np.float32)
     u = g.uniform(-u_bound, u_bound, size=C).astype(np.float32)
     shape = (B, T, C)
-    k64 = g.normal(0.0, k_std, size=shape)
-    v64 = g.standard_normal(size=shape)
-    r64 = g.standard_normal(size=shape)
-    dy = g.standard_normal(size=shape).astype(np.float32) if with_dy else None
+    f32 = np.float32
+    k32 = g.standard_normal(size=shape, dtype=f32)
+    if k_std != 1.0:
+        k32 *= f32(k_std)
+    v32 = g.standard_normal(size=shape, dtype=f32)
+    r32 = g.standard_normal(size=shape, dtype=f32)
+    dy = g.standard_normal(size=shape, dtype=f32) if with_dy else None
     if spike_frac > 0.0:
-        mask = g.random(size=shape) < spike_frac
-        k64[mask] = spike_value
+        mask = g.random(size=shape, dtype=f32) < f32(spike_frac)
+        k32[mask] = f32(spike_value)
         del mask
     out = WkvInputs(B, T, C, dtype, w, u, None, None, None, dy)
-    for name, x64 in (("k", k64), ("v", v64), ("r", r64)):
-        x, bits = _store(x64, dtype)
+    for name, x32 in (("k", k32), ("v", v32), ("r", r32)):
+        x, bits = _store(x32, dtype)
         setattr(out, name, x)
         if bits is not None:
             out.bits[name] = bits
@@ -135,10 +143,12 @@ class DecodeInputs:
     seed: int
 
     def step(self, s: int):
-        """k, v, r for step s, each [N, L, C] float32; step s has its own stream."""
+        """k, v, r for step s, each [N, L, C] float32; step s has its own stream
+        (PCG64 seeded with [seed, 1 + s]) and draws float32 normals directly, so that the
+        64 chained steps of the full workload can be generated quickly."""
         g = np.random.Generator(np.random.PCG64([self.seed, 1 + s]))
         shape = (self.N, self.L, self.C)
-        return tuple(g.standard_normal(size=shape).astype(np.float32) for _ in range(3))
+        return tuple(g.standard_normal(size=shape, dtype=np.float32) for _ in range(3))
 
 
 def decode_batch(seed: int = 0, N: int = 256, L: int = 32, C: int = 4096) -> DecodeInputs:
