@@ -33,7 +33,6 @@ sys.path.insert(0, ROOT)
 METRIC = "WKV fwd G(B·T·C)/s and HBM GB/s vs B200 peak at B=8,T=4096,C=4096"
 UNIT = "G(B·T·C)/s"
 B, T, C = 8, 4096, 4096
-ELEMS = B * T * C
 BYTES_PER_ELEM = 8          # read k, v, r and write y, 2 bytes each
 FALLBACK_HBM_GBS = 6650.0
 KERNEL = "wkv_fwd_tma_kernel<bf16, gate>"
@@ -226,7 +225,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    x = wkv_inputs.long_bf16(seed=rank)
+    Bn = args.batch
+    ELEMS = Bn * T * C
+    x = wkv_inputs.long_bf16(seed=rank, B=Bn)
 
     def to_bf16(bits, pin=False):
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
@@ -313,17 +314,17 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         rate, rows = cpu_oracle_rate(x, budget_s=10.0)
         cpu = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{rows} of 8 batch rows ({rows} x 4096 x 4096 elements) of the same "
-                         f"inputs, fp64 recurrence, 1 thread"}
+               "sample": f"{rows} of {Bn} batch rows ({rows} x 4096 x 4096 elements) of the "
+                         f"same inputs, fp64 recurrence, 1 thread"}
     clocks = sampler.summary()
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": "WKV forward bf16 in/out, B=8 T=4096 C=4096 (7B-shaped, "
+        "config": {"workload": f"WKV forward bf16 in/out, B={Bn} T=4096 C=4096 (7B-shaped, "
                                "k spikes of +60), one batch per GPU",
-                   "B": B, "T": T, "C": C, "storage": "bf16", "global_batch": B * world,
+                   "B": Bn, "T": T, "C": C, "storage": "bf16", "global_batch": Bn * world,
                    "seq_len": T, "parallelism": f"dp{world} (independent batches)",
                    "l2": "inputs 805 MB + output 268 MB per step > 126 MB L2; no flush",
                    "kernel": KERNEL},
@@ -349,6 +350,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=B,
+                    help="batch rows per GPU (default 8, the measured workload; smaller "
+                         "values are for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -123,6 +123,26 @@ WKV_API int wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, con
                             float* b, float* p, cudaStream_t stream);
 
 /*
+ * Backward of the forward (wkv_forward with the same w, u, k, v, r), fp32: gradients of
+ * L = sum dy . y. The pages say only that the operator trains by ordinary backpropagation
+ * (news page "RWKV CUDA linear attention GPU": fused forward and backward kernels); the
+ * formulas are the chain rule applied to the wkv_t equation of the concept page, section
+ * 3.2, with w the positive decay rate itself:
+ *   dk, dv, dr: fp32 (B, T, C), overwritten; dr = dL/dr, may be NULL (then not computed);
+ *   dw, du:     fp32 [C], overwritten with the sums over b and t.
+ * r == NULL: the ungated forward (y = wkv); dr must then be NULL.
+ * workspace: caller-owned device memory of at least wkv_backward_workspace_bytes(B, T, C)
+ * bytes, 256-byte aligned; its contents need no initialisation and are scratch after the
+ * call. Too small a workspace returns WKV_ERR_INVALID_ARG. Deterministic: dw and du are
+ * reduced over b in a fixed order.
+ */
+WKV_API size_t wkv_backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
+WKV_API int wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                         const float* k, const float* v, const float* r, const float* dy,
+                         float* dk, float* dv, float* dw, float* du, float* dr, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Query and clear device-side errors. Synchronises `stream`, then returns WKV_ERR_TIMEOUT
  * if any kernel of this library on the current device gave up a bounded wait since the
  * last query (the outputs of that call are then undefined), WKV_ERR_CUDA if the stream

@@ -32,6 +32,15 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
                                       const float* u, const void* k, const void* v,
                                       const void* r, void* y, int bf16, cudaStream_t stream);
 
+/*
+ * Forces the backward's plain (non-TMA) tile movement; otherwise as wkv_backward.
+ */
+WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const float* w,
+                                       const float* u, const float* k, const float* v,
+                                       const float* r, const float* dy, float* dk, float* dv,
+                                       float* dw, float* du, float* dr, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

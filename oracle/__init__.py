@@ -52,7 +52,7 @@ def _load():
         lib.oracle_wkv_direct.argtypes = [I, I, I] + [P] * 8
         lib.oracle_wkv_recurrent.argtypes = [I, I, I] + [P] * 10
         lib.oracle_wkv_decode.argtypes = [I, I, I] + [P] * 8
-        lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 11
+        lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 13
         for f in (lib.oracle_wkv_direct, lib.oracle_wkv_recurrent, lib.oracle_wkv_decode,
                   lib.oracle_wkv_backward):
             f.restype = ctypes.c_int
@@ -110,7 +110,8 @@ def wkv_decode(w, u, k, v, r, A, Bd):
 
 
 def wkv_backward(w, u, k, v, r, dy):
-    """Analytic fp64 gradients. Returns dict dk, dv, dw, du, dr (dr None if r is None)."""
+    """Analytic fp64 gradients. Returns dict dk, dv, dw, du, dr (dr None if r is None),
+    and dw_abs, du_abs: the sums of |term| behind dw and du."""
     w, u, k, v, r, dy = map(_f64, (w, u, k, v, r, dy))
     B, T, C = k.shape
     dk = np.empty((B, T, C))
@@ -118,10 +119,12 @@ def wkv_backward(w, u, k, v, r, dy):
     dr = np.empty((B, T, C)) if r is not None else None
     dw = np.empty(C)
     du = np.empty(C)
+    dwa = np.empty(C)
+    dua = np.empty(C)
     _check(_load().oracle_wkv_backward(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
                                        _ptr(dy), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
-                                       _ptr(dr)))
-    return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr}
+                                       _ptr(dr), _ptr(dwa), _ptr(dua)))
+    return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dw_abs": dwa, "du_abs": dua}
 
 
 def state_from_scaled(a, b, p):

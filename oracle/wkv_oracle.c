@@ -143,18 +143,26 @@ int oracle_wkv_decode(int64_t N, int64_t L, int64_t C, const double *w, const do
  * computed by the reverse recurrences beta_{i-1} = h_i + e^{-w} beta_i and
  * betad_{i-1} = e^{-w} (betad_i + beta_i) (and the same for gamma).
  * r == NULL: no gate (g_t = dy_t) and dr is not written. dr may be NULL.
- * dw, du [C] are overwritten with the sums over b and t.
+ * dw, du [C] are overwritten with the sums over b and t. dw_abs, du_abs [C] (may be NULL)
+ * receive the sums of the absolute values of the same terms, the scale against which a
+ * float reduction's rounding is judged.
  */
 int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
                         const double *k, const double *v, const double *r, const double *dy,
-                        double *dk, double *dv, double *dw, double *du, double *dr)
+                        double *dk, double *dv, double *dw, double *du, double *dr,
+                        double *dw_abs, double *du_abs)
 {
     if (B < 0 || T < 0 || C < 0 || !w || !u || !k || !v || !dy || !dk || !dv || !dw || !du)
         return -1;
     double *wkv = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
     double *D = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
     if (!wkv || !D) { free(wkv); free(D); return -1; }
-    for (int64_t c = 0; c < C; ++c) { dw[c] = 0.0; du[c] = 0.0; }
+    for (int64_t c = 0; c < C; ++c) {
+        dw[c] = 0.0;
+        du[c] = 0.0;
+        if (dw_abs) dw_abs[c] = 0.0;
+        if (du_abs) du_abs[c] = 0.0;
+    }
     for (int64_t b = 0; b < B; ++b)
         for (int64_t c = 0; c < C; ++c) {
             double decay = exp(-w[c]), eu = exp(u[c]);
@@ -169,7 +177,7 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
                 d = decay * d + ek;
             }
             double beta = 0.0, gamma = 0.0, betad = 0.0, gammad = 0.0;
-            double dwc = 0.0, duc = 0.0;
+            double dwc = 0.0, duc = 0.0, dwa = 0.0, dua = 0.0;
             for (int64_t i = T - 1; i >= 0; --i) {           /* reverse */
                 double ki = k[AT(b, i, c)], vi = v[AT(b, i, c)], dyi = dy[AT(b, i, c)];
                 double s = r ? sigm(r[AT(b, i, c)]) : 1.0;
@@ -177,8 +185,12 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
                 double ek = exp(ki);
                 dv[AT(b, i, c)] = ek * (h * eu + beta);
                 dk[AT(b, i, c)] = ek * (h * eu * (vi - wkv[i]) + vi * beta - gamma);
-                dwc += -ek * (vi * betad - gammad);
-                duc += h * eu * ek * (vi - wkv[i]);
+                double tw = -ek * (vi * betad - gammad);
+                double tu = h * eu * ek * (vi - wkv[i]);
+                dwc += tw;
+                duc += tu;
+                dwa += fabs(tw);
+                dua += fabs(tu);
                 if (r && dr) dr[AT(b, i, c)] = dyi * wkv[i] * s * (1.0 - s);
                 betad = decay * (betad + beta);
                 gammad = decay * (gammad + gamma);
@@ -187,6 +199,8 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
             }
             dw[c] += dwc;
             du[c] += duc;
+            if (dw_abs) dw_abs[c] += dwa;
+            if (du_abs) du_abs[c] += dua;
         }
     free(wkv);
     free(D);

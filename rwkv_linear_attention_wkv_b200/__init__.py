@@ -12,7 +12,8 @@ import ctypes
 import os
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
-           "wkv_stream_status", "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
+           "wkv_backward", "wkv_backward_workspace_bytes", "wkv_stream_status",
+           "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
 
@@ -33,6 +34,10 @@ _SIGS = {
     "wkv_forward_state": ([_I, _I, _I] + [_P] * 12 + [_P], ctypes.c_int),
     "wkv_decode_step": ([_I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
     "wkv_stream_status": ([_P], ctypes.c_int),
+    "wkv_backward_workspace_bytes": ([_I, _I, _I], ctypes.c_size_t),
+    "wkv_backward": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "wkv_testing_backward_plain": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P],
+                                   ctypes.c_int),
     "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
     "wkv_testing_forward_plain": ([_I, _I, _I] + [_P] * 6 + [ctypes.c_int, _P], ctypes.c_int),
 }
@@ -170,6 +175,54 @@ def wkv_decode_step(w, u, k, v, r, a, b, p, y=None, stream=None):
     _call("wkv_decode_step", N, L, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
           _ptr(a), _ptr(b), _ptr(p), _stream(stream))
     return y
+
+
+def wkv_backward_workspace_bytes(B: int, T: int, C: int) -> int:
+    return int(lib.wkv_backward_workspace_bytes(B, T, C))
+
+
+def wkv_backward(w, u, k, v, r, dy, want_dr=True, workspace=None, out=None, stream=None,
+                 _entry="wkv_backward"):
+    """fp32 gradients of sum(dy * y) for y = wkv_forward(w, u, k, v, r).
+
+    Returns a dict with dk, dv (B, T, C), dw, du (C,) and dr (B, T, C; None when r is None
+    or want_dr is False). `workspace` (uint8 CUDA tensor of at least
+    wkv_backward_workspace_bytes(B, T, C) bytes) is allocated when not given; `out` may
+    hold preallocated dk, dv, dw, du, dr tensors.
+    """
+    torch = _torch()
+    f32 = torch.float32
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    _need(k, "k", f32)
+    for n, t in (("v", v), ("dy", dy)):
+        _need(t, n, f32, (B, T, C))
+    if r is not None:
+        _need(r, "r", f32, (B, T, C))
+    _need(w, "w", f32, (C,))
+    _need(u, "u", f32, (C,))
+    out = dict(out or {})
+    dev = k.device
+    for n, shape in (("dk", (B, T, C)), ("dv", (B, T, C)), ("dw", (C,)), ("du", (C,))):
+        if out.get(n) is None:
+            out[n] = torch.empty(shape, dtype=f32, device=dev)
+        _need(out[n], n, f32, shape)
+    if r is not None and want_dr:
+        if out.get("dr") is None:
+            out["dr"] = torch.empty((B, T, C), dtype=f32, device=dev)
+        _need(out["dr"], "dr", f32, (B, T, C))
+    else:
+        out["dr"] = None
+    nbytes = wkv_backward_workspace_bytes(B, T, C)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA tensor of at least {nbytes} bytes")
+    _call(_entry, B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(dy),
+          _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dw"]), _ptr(out["du"]), _ptr(out["dr"]),
+          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return out
 
 
 def wkv_stream_status(stream=None) -> int:

@@ -121,6 +121,36 @@ static int forward_impl(int64_t B, int64_t T, int64_t C, const float* w, const f
   return launch_fwd_stream(a, bf16, /*force_plain=*/T == 0, stream);
 }
 
+static int backward_impl(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                         const float* k, const float* v, const float* r, const float* dy,
+                         float* dk, float* dv, float* dw, float* du, float* dr, void* workspace,
+                         size_t workspace_bytes, bool force_plain, cudaStream_t stream) {
+  if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  if (C == 0) return WKV_OK;
+  if (!w || !u || !dw || !du) return WKV_ERR_INVALID_ARG;
+  if (r == nullptr && dr != nullptr) return WKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {w, u, k, v, r, dy, dk, dv, dw, du, dr};
+  for (const void* q : ptrs)
+    if (!aligned(q, 4)) return WKV_ERR_ALIGNMENT;
+  if (B == 0 || T == 0) {  // no tokens: zero gradients for the parameters
+    if (cudaMemsetAsync(dw, 0, size_t(C) * sizeof(float), stream) != cudaSuccess ||
+        cudaMemsetAsync(du, 0, size_t(C) * sizeof(float), stream) != cudaSuccess)
+      return WKV_ERR_CUDA;
+    return WKV_OK;
+  }
+  if (!k || !v || !dy || !dk || !dv) return WKV_ERR_INVALID_ARG;
+  if (T >= (int64_t(1) << 31) || C >= (int64_t(1) << 31) || B >= (int64_t(1) << 31) ||
+      B > INT64_MAX / T / C || B * ((C + 31) / 32) >= (int64_t(1) << 31))
+    return WKV_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 256) ||
+      workspace_bytes < backward_workspace_bytes(B, T, C))
+    return WKV_ERR_INVALID_ARG;
+  unsigned* err = error_word();
+  if (err == nullptr) return WKV_ERR_CUDA;
+  BwdArgs a{B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace, err};
+  return launch_backward(a, force_plain, stream);
+}
+
 }  // namespace wkv
 
 using namespace wkv;
@@ -174,6 +204,19 @@ WKV_API int wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, con
   if (L > INT64_MAX / C || N > INT64_MAX / (L * C)) return WKV_ERR_UNSUPPORTED;
   DecodeArgs d{N, L, C, w, u, k, v, r, y, a, b, p};
   return launch_decode(d, stream);
+}
+
+WKV_API size_t wkv_backward_workspace_bytes(int64_t B, int64_t T, int64_t C) {
+  if (B <= 0 || T <= 0 || C <= 0) return 256;
+  return backward_workspace_bytes(B, T, C);
+}
+
+WKV_API int wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                         const float* k, const float* v, const float* r, const float* dy,
+                         float* dk, float* dv, float* dw, float* du, float* dr, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
+                       workspace_bytes, false, stream);
 }
 
 WKV_API int wkv_stream_status(cudaStream_t stream) {
@@ -230,6 +273,15 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
   if (err == nullptr) return WKV_ERR_CUDA;
   FwdArgs a{B, T, C, w, u, k, v, r, y, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, err};
   return launch_fwd_stream(a, bf16 != 0, /*force_plain=*/true, stream);
+}
+
+WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const float* w,
+                                       const float* u, const float* k, const float* v,
+                                       const float* r, const float* dy, float* dk, float* dv,
+                                       float* dw, float* du, float* dr, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream) {
+  return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
+                       workspace_bytes, true, stream);
 }
 
 }  // extern "C"

@@ -18,10 +18,11 @@
 namespace wkv {
 
 // Process n tokens of a tile already in shared memory (rows of 32 elements, this lane's
-// column), in windows of RB tokens. FULL: n == TT, fully unrolled.
+// column), in windows of RB tokens. FULL: n == TT, fully unrolled; otherwise the window
+// length is the runtime value rb.
 template <typename Tin, bool GATE, bool FASTOUT, int TT, int RB, bool FULL>
 __device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, const Tin* K,
-                                            const Tin* V, const Tin* R, Tin* Y, int n) {
+                                            const Tin* V, const Tin* R, Tin* Y, int n, int rb) {
   if (FULL) {
 #pragma unroll
     for (int w0 = 0; w0 < TT; w0 += RB) {
@@ -43,16 +44,33 @@ __device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, 
       const float v = Elem<Tin>::to_f(V[row]);
       const float r = GATE ? Elem<Tin>::to_f(R[row]) : 0.f;
       Y[row] = Elem<Tin>::from_f(wkv_token<GATE, FASTOUT>(s, cp, float(j + 1), k, v, r));
-      if (++j == RB) {
-        wkv_rebase(s, float(RB) * cp.w2);
+      if (++j == rb) {
+        wkv_rebase(s, float(rb) * cp.w2);
         j = 0;
       }
     }
-    if (j) wkv_rebase(s, float(j) * cp.w2);
+    if (j) wkv_rebase_partial(s, j, cp.w2);
   }
 }
 
-template <typename Tin, bool GATE, int TT, int S, int RB>
+template <typename Tin, bool GATE, bool FASTOUT, int TT>
+__device__ __forceinline__ void full_tile(ChanState& s, const ChanParams& cp, const Tin* K,
+                                          const Tin* V, const Tin* R, Tin* Y, int rb) {
+  if (rb == 16)
+    tile_tokens<Tin, GATE, FASTOUT, TT, 16, true>(s, cp, K, V, R, Y, TT, rb);
+  else if (rb == 4)
+    tile_tokens<Tin, GATE, FASTOUT, TT, 4, true>(s, cp, K, V, R, Y, TT, rb);
+  else
+    tile_tokens<Tin, GATE, FASTOUT, TT, 1, true>(s, cp, K, V, R, Y, TT, rb);
+}
+
+// Largest window allowed for the output precision (see window_tokens).
+template <typename Tin>
+constexpr float window_limit() {
+  return sizeof(Tin) == 2 ? 512.f : 128.f;
+}
+
+template <typename Tin, bool GATE, int TT, int S>
 __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_y, int T,
@@ -102,6 +120,7 @@ __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
   const bool has_state = a0 != nullptr;
   ChanState s = (has_state && valid) ? load_state(a0[sidx], b0[sidx], p0[sidx]) : empty_state();
   const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+  const int rb = window_tokens(cp.w2, window_limit<Tin>());
 
   for (int i = 0; i < ntiles; ++i) {
     const int st = i % S;
@@ -115,14 +134,14 @@ __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
     const int n = min(TT, T - i * TT);
     if (n == TT) {
       if (fast)
-        tile_tokens<Tin, GATE, true, TT, RB, true>(s, cp, K, V, R, Y, n);
+        full_tile<Tin, GATE, true, TT>(s, cp, K, V, R, Y, rb);
       else
-        tile_tokens<Tin, GATE, false, TT, RB, true>(s, cp, K, V, R, Y, n);
+        full_tile<Tin, GATE, false, TT>(s, cp, K, V, R, Y, rb);
     } else {
       if (fast)
-        tile_tokens<Tin, GATE, true, TT, RB, false>(s, cp, K, V, R, Y, n);
+        tile_tokens<Tin, GATE, true, TT, 1, false>(s, cp, K, V, R, Y, n, rb);
       else
-        tile_tokens<Tin, GATE, false, TT, RB, false>(s, cp, K, V, R, Y, n);
+        tile_tokens<Tin, GATE, false, TT, 1, false>(s, cp, K, V, R, Y, n, rb);
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -142,7 +161,7 @@ __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
 }
 
 // Plain kernel: one thread per (b, c), coalesced across threads, no shared memory.
-template <typename Tin, bool GATE, int RB>
+template <typename Tin, bool GATE>
 __global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
     int64_t B, int64_t T, int64_t C, const float* __restrict__ w, const float* __restrict__ u,
     const Tin* __restrict__ k, const Tin* __restrict__ v, const Tin* __restrict__ r,
@@ -156,6 +175,7 @@ __global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
   const bool has_state = a0 != nullptr;
   ChanState s = (has_state && valid) ? load_state(a0[idx], b0[idx], p0[idx]) : empty_state();
   const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+  const int rb = window_tokens(cp.w2, window_limit<Tin>());
   if (!valid) return;
   const int64_t base = bb * T * C + c;
   int j = 0;
@@ -167,12 +187,12 @@ __global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
     const float out = fast ? wkv_token<GATE, true>(s, cp, float(j + 1), kk, vv, rr)
                            : wkv_token<GATE, false>(s, cp, float(j + 1), kk, vv, rr);
     y[e] = Elem<Tin>::from_f(out);
-    if (++j == RB) {
-      wkv_rebase(s, float(RB) * cp.w2);
+    if (++j == rb) {
+      wkv_rebase(s, float(rb) * cp.w2);
       j = 0;
     }
   }
-  if (j) wkv_rebase(s, float(j) * cp.w2);
+  if (j) wkv_rebase_partial(s, j, cp.w2);
   if (a1 != nullptr) {
     a1[idx] = s.a;
     b1[idx] = s.b;
@@ -186,7 +206,6 @@ __global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
 namespace {
 
 constexpr int kTT = 32;   // tokens per tile
-constexpr int kRB = 16;   // tokens per log-scale window
 
 template <typename Tin>
 constexpr int stages() {
@@ -209,7 +228,7 @@ int launch_tma(const FwdArgs& a, cudaStream_t stream) {
   if (!rc) rc = encode_btc_map(&tr, GATE ? a.r : a.k, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
   if (!rc) rc = encode_btc_map(&ty, a.y, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
   if (rc) return rc;
-  auto kern = wkv_fwd_tma_kernel<Tin, GATE, kTT, stages<Tin>(), kRB>;
+  auto kern = wkv_fwd_tma_kernel<Tin, GATE, kTT, stages<Tin>()>;
   const size_t smem = tma_smem_bytes<Tin, GATE>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
@@ -226,7 +245,7 @@ int launch_plain(const FwdArgs& a, cudaStream_t stream) {
   const int64_t n = a.B * a.C;
   const int block = 128;
   const int64_t grid = (n + block - 1) / block;
-  wkv_fwd_plain_kernel<Tin, GATE, kRB><<<unsigned(grid), block, 0, stream>>>(
+  wkv_fwd_plain_kernel<Tin, GATE><<<unsigned(grid), block, 0, stream>>>(
       a.B, a.T, a.C, a.w, a.u, static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
       static_cast<const Tin*>(a.r), static_cast<Tin*>(a.y), a.a0, a.b0, a.p0, a.a1, a.b1, a.p1);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;

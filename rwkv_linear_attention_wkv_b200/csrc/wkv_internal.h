@@ -68,4 +68,25 @@ struct DecodeArgs {
 };
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// Backward over (B, T, C), fp32. r null: no gate (dr must be null). ws: device workspace of
+// backward_workspace_bytes(B, T, C) bytes, 256-byte aligned; no part needs clearing.
+struct BwdArgs {
+  int64_t B, T, C;
+  const float* w;
+  const float* u;
+  const float* k;
+  const float* v;
+  const float* r;
+  const float* dy;
+  float* dk;
+  float* dv;
+  float* dw;
+  float* du;
+  float* dr;
+  void* ws;
+  unsigned* err;
+};
+size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
+int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);
+
 }  // namespace wkv

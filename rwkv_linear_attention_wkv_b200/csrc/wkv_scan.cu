@@ -32,7 +32,6 @@ namespace {
 
 constexpr int kW = 8;        // warps per CTA (sub-chunks per segment)
 constexpr int kLS = 32;      // tokens per sub-chunk
-constexpr int kRB = 16;      // tokens per log-scale window
 constexpr int kSeg = kW * kLS;
 // Fewer channels than this leave the streaming kernel without enough warps per SM.
 constexpr int64_t kChunkBelowChannels = 148 * 32 * 4;
@@ -46,7 +45,7 @@ __device__ __forceinline__ Agg agg_empty() { return Agg{0.f, 0.f, kEmptyLogScale
 // X (+) Y where Y spans `len` tokens after X.
 __device__ __forceinline__ Agg combine(const Agg& X, const Agg& Y, float len, float w2) {
   float xh, xl;
-  two_sum(X.ph, X.pl - len * w2, xh, xl);
+  decay_pair(X.ph, X.pl, len, w2, xh, xl);
   const float d = (xh - Y.ph) + (xl - Y.pl);
   const float f = ex2(-fabsf(d));
   Agg r;
@@ -160,18 +159,19 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   float* Y = sk + warp * kTile + lane;
 
   // ---- 1. sub-chunk aggregate from the empty state ----
+  const int rb = window_tokens(cp.w2, 128.f);
   if (n > 0) mbar_wait(bar, 0, err);
   ChanState s = empty_state();
   {
     int j = 0;
     for (int t = 0; t < n; ++t) {
       wkv_absorb(s, cp, float(j + 1), K[t * 32], V[t * 32]);
-      if (++j == kRB) {
-        wkv_rebase(s, float(kRB) * cp.w2);
+      if (++j == rb) {
+        wkv_rebase(s, float(rb) * cp.w2);
         j = 0;
       }
     }
-    if (j) wkv_rebase(s, float(j) * cp.w2);
+    if (j) wkv_rebase_partial(s, j, cp.w2);
   }
   const Agg mine = to_agg(s);
   sagg[warp * 32 + lane] = make_float4(mine.a, mine.b, mine.ph, mine.pl);
@@ -257,12 +257,12 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
       const float kk = K[t * 32], vv = V[t * 32], rr = GATE ? R[t * 32] : 0.f;
       Y[t * 32] = fast ? wkv_token<GATE, true>(s, cp, float(j + 1), kk, vv, rr)
                        : wkv_token<GATE, false>(s, cp, float(j + 1), kk, vv, rr);
-      if (++j == kRB) {
-        wkv_rebase(s, float(kRB) * cp.w2);
+      if (++j == rb) {
+        wkv_rebase(s, float(rb) * cp.w2);
         j = 0;
       }
     }
-    if (j) wkv_rebase(s, float(j) * cp.w2);
+    if (j) wkv_rebase_partial(s, j, cp.w2);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {

@@ -16,7 +16,11 @@
 //   * at the end of the window P = Q + pl - n w2 is re-split exactly (TwoSum).
 // Decaying the scale by w2 once per token in float would round the same way every step
 // (the low bits of w2 below ulp(P) are constant) and drift by up to ulp(P)/2 per token;
-// the window form rounds each m_j once and never accumulates.
+// the window form rounds each m_j once and never accumulates. The price is that m_j and Q
+// grow to about n w2 within a window, and their difference d is rounded at that magnitude;
+// so the window length n is chosen per warp from the largest w2 of its channels
+// (window_tokens below): long windows for slowly decaying channels, where drift matters,
+// short ones for fast decay, where only the last few tokens carry weight.
 //
 // Per token (d = m_j - Q; one of e1, e2 is 1, the other 2^{-|d|}):
 //   state update   a' = e1 a + e2 v,  b' = e1 b + e2,  Q' = max(Q, m_j)
@@ -129,13 +133,41 @@ __device__ __forceinline__ void wkv_absorb(ChanState& s, const ChanParams& cp, f
   s.b = fmaf(e1, s.b, e2);
 }
 
-// End of a window of n tokens: P = Q + pl - n w2, re-split exactly.
+// End of a window of n tokens: P = Q + pl - n w2, re-split exactly. For n a power of two
+// n w2 is exact; the one rounding of pl - n w2 is 2^-24 of the window's decay, the same
+// relative size as the rounding of w2 itself, and does not grow with the window count.
 __device__ __forceinline__ void wkv_rebase(ChanState& s, float nw2) {
   const float c2 = s.pl - nw2;
   float hi, lo;
   two_sum(s.Q, c2, hi, lo);
   s.Q = hi;
   s.pl = lo;
+}
+
+// (h, l) = ph + pl - n w2 as an unevaluated pair, with the product n w2 taken exactly
+// (its rounding error recovered by an fma) and the large subtraction done by TwoSum.
+// For spans that are not a power of two (partial windows, carries across chunks).
+__device__ __forceinline__ void decay_pair(float ph, float pl, float n, float w2, float& h,
+                                           float& l) {
+  const float prod = n * w2;
+  const float perr = fmaf(n, w2, -prod);  // n w2 = prod + perr exactly
+  float h1, l1;
+  two_sum(ph, -prod, h1, l1);
+  two_sum(h1, l1 + (pl - perr), h, l);
+}
+
+__device__ __forceinline__ void wkv_rebase_partial(ChanState& s, int n, float w2) {
+  decay_pair(s.Q, s.pl, float(n), w2, s.Q, s.pl);
+}
+
+// Window length for a warp: the largest of 16, 4, 1 tokens for which n w2 stays within
+// `limit` (log2 units) for every channel of the warp. fp32 outputs use limit 128 (m_j
+// rounded at ~2^-17 absolute), bf16 outputs 512 (bf16 resolution is 2^-8 relative).
+__device__ __forceinline__ int window_tokens(float w2, float limit) {
+  float m = w2;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return (16.f * m <= limit) ? 16 : ((4.f * m <= limit) ? 4 : 1);
 }
 
 }  // namespace wkv

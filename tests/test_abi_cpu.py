@@ -1,0 +1,89 @@
+"""Host-side checks of the C-ABI library that need no GPU: it loads, exports every symbol
+the headers declare, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def W():
+    import rwkv_linear_attention_wkv_b200 as W
+    return W
+
+
+def declared_symbols():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"WKV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+    return names
+
+
+def test_library_exports_every_declared_symbol(W):
+    names = declared_symbols()
+    assert "wkv_forward" in names and "wkv_backward" in names and len(names) >= 10
+    for n in names:
+        assert hasattr(W.lib, n), n
+
+
+def test_status_strings(W):
+    assert [W.wkv_status_string(i) for i in range(6)] == [
+        "WKV_OK", "WKV_ERR_INVALID_ARG", "WKV_ERR_ALIGNMENT", "WKV_ERR_CUDA",
+        "WKV_ERR_TIMEOUT", "WKV_ERR_UNSUPPORTED"]
+    assert W.wkv_status_string(99) == "WKV_ERR_UNKNOWN"
+    assert W.lib.wkv_version() >= 10000
+
+
+def P(x):
+    return ctypes.c_void_p(x)
+
+
+def test_forward_argument_checks(W):
+    f = W.lib.wkv_forward
+    ok = P(4096)
+    assert f(-1, 1, 1, ok, ok, ok, ok, ok, ok, None) == 1
+    assert f(1, -1, 1, ok, ok, ok, ok, ok, ok, None) == 1
+    assert f(1, 1, 1, None, ok, ok, ok, ok, ok, None) == 1      # w missing
+    assert f(1, 1, 1, ok, ok, None, ok, ok, ok, None) == 1      # k missing
+    assert f(1, 1, 1, ok, ok, ok, ok, None, None, None) == 1    # y missing
+    assert f(1, 1, 4, ok, ok, P(4098), ok, None, ok, None) == 2  # k not 4-byte aligned
+    assert f(0, 5, 5, None, None, None, None, None, None, None) == 0   # empty
+    assert f(5, 5, 0, None, None, None, None, None, None, None) == 0
+    assert f(1, 1 << 31, 4, ok, ok, ok, ok, ok, ok, None) == 5       # T too large
+    g = W.lib.wkv_forward_bf16
+    assert g(1, 1, 8, ok, ok, P(4097), ok, None, ok, None) == 2      # bf16 needs 2-byte
+    st = W.lib.wkv_forward_state
+    # state pointers must come as a full triple
+    assert st(1, 1, 4, ok, ok, ok, ok, None, ok, ok, None, None, None, None, None, None) == 1
+    assert st(1, 1, 4, ok, ok, ok, ok, None, ok, None, None, None, ok, ok, None, None) == 1
+
+
+def test_decode_and_backward_argument_checks(W):
+    ok = P(4096)
+    d = W.lib.wkv_decode_step
+    assert d(-1, 1, 1, *([ok] * 9), None) == 1
+    assert d(1, 1, 1, ok, ok, ok, ok, None, ok, ok, ok, None, None) == 1   # p missing
+    assert d(0, 4, 4, *([None] * 9), None) == 0
+    assert d(1, 1, 1, ok, ok, P(4099), ok, None, ok, ok, ok, ok, None) == 2
+    bw = W.lib.wkv_backward
+    need = W.wkv_backward_workspace_bytes(2, 64, 32)
+    args = [ok] * 5 + [ok] * 6
+    assert bw(2, 64, 32, *args, ok, need - 1, None) == 1                    # too small
+    assert bw(2, 64, 32, *args, P(4096 + 128), need, None) == 1             # not 256-aligned
+    assert bw(2, 64, 32, ok, ok, ok, ok, None, ok, ok, ok, ok, ok, ok, ok, need, None) == 1
+    assert bw(-2, 64, 32, *args, ok, need, None) == 1
+
+
+def test_backward_workspace_size(W):
+    # checkpoints (a, b, Q, pl) per 32-token chunk and channel, plus dw, du partials [B, C]
+    def a256(x):
+        return (x + 255) // 256 * 256
+    for B, T, C in ((16, 1024, 768), (1, 33, 5), (3, 1, 4096)):
+        nch = (T + 31) // 32
+        want = a256(B * nch * C * 16) + 2 * a256(B * C * 4)
+        assert W.wkv_backward_workspace_bytes(B, T, C) == want

@@ -232,6 +232,7 @@ def test_backward_matches_central_differences(gate):
             assert fd("r", r, idx) == pytest.approx(g["dr"][idx], rel=1e-6, abs=1e-8)
     else:
         assert g["dr"] is None
+    assert np.all(g["dw_abs"] >= np.abs(g["dw"])) and np.all(g["du_abs"] >= np.abs(g["du"]))
 
 
 def test_spike_inputs_stay_finite_and_in_range():
