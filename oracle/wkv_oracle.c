@@ -144,8 +144,11 @@ int oracle_wkv_decode(int64_t N, int64_t L, int64_t C, const double *w, const do
  * betad_{i-1} = e^{-w} (betad_i + beta_i) (and the same for gamma).
  * r == NULL: no gate (g_t = dy_t) and dr is not written. dr may be NULL.
  * dw, du [C] are overwritten with the sums over b and t. dw_abs, du_abs [C] (may be NULL)
- * receive the sums of the absolute values of the same terms, the scale against which a
- * float reduction's rounding is judged.
+ * receive the scale against which a float computation of them is judged: the sums of the
+ * absolute values of the terms of their full expansion,
+ *   dw = -sum_{i<t} (t-1-i) e^{k_i-(t-1-i)w} h_t v_i + sum_{i<t} (t-1-i) e^{k_i-(t-1-i)w} h_t wkv_t,
+ *   du =  sum_t h_t e^{u+k_t} v_t - sum_t h_t e^{u+k_t} wkv_t,
+ * accumulated by the same recurrences run on |h_t|, |v_i|, |wkv_t|.
  */
 int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
                         const double *k, const double *v, const double *r, const double *dy,
@@ -177,6 +180,7 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
                 d = decay * d + ek;
             }
             double beta = 0.0, gamma = 0.0, betad = 0.0, gammad = 0.0;
+            double abeta = 0.0, agamma = 0.0, abetad = 0.0, agammad = 0.0;
             double dwc = 0.0, duc = 0.0, dwa = 0.0, dua = 0.0;
             for (int64_t i = T - 1; i >= 0; --i) {           /* reverse */
                 double ki = k[AT(b, i, c)], vi = v[AT(b, i, c)], dyi = dy[AT(b, i, c)];
@@ -185,17 +189,19 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
                 double ek = exp(ki);
                 dv[AT(b, i, c)] = ek * (h * eu + beta);
                 dk[AT(b, i, c)] = ek * (h * eu * (vi - wkv[i]) + vi * beta - gamma);
-                double tw = -ek * (vi * betad - gammad);
-                double tu = h * eu * ek * (vi - wkv[i]);
-                dwc += tw;
-                duc += tu;
-                dwa += fabs(tw);
-                dua += fabs(tu);
+                dwc += -ek * (vi * betad - gammad);
+                duc += h * eu * ek * (vi - wkv[i]);
+                dwa += ek * (fabs(vi) * abetad + agammad);
+                dua += fabs(h) * eu * ek * (fabs(vi) + fabs(wkv[i]));
                 if (r && dr) dr[AT(b, i, c)] = dyi * wkv[i] * s * (1.0 - s);
                 betad = decay * (betad + beta);
                 gammad = decay * (gammad + gamma);
                 beta = h + decay * beta;
                 gamma = h * wkv[i] + decay * gamma;
+                abetad = decay * (abetad + abeta);
+                agammad = decay * (agammad + agamma);
+                abeta = fabs(h) + decay * abeta;
+                agamma = fabs(h * wkv[i]) + decay * agamma;
             }
             dw[c] += dwc;
             du[c] += duc;

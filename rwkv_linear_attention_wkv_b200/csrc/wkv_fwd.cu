@@ -17,25 +17,50 @@
 
 namespace wkv {
 
+// One full window of RB tokens from shared memory, written in phases so that the only
+// serial chains are the ones the recurrence has (a running max for the scale, one fma per
+// token for a and b): every load of the window first, then the log-weights and their
+// running max, then the per-token arithmetic, then every store. (Token by token, each
+// token's loads would wait for the previous token's store, which the compiler must assume
+// may alias them.)
+template <typename Tin, bool GATE, bool FASTOUT, int RB>
+__device__ __forceinline__ void window_tokens_smem(ChanState& s, const ChanParams& cp,
+                                                   const Tin* K, const Tin* V, const Tin* R,
+                                                   Tin* Y) {
+  float kk[RB], vv[RB], rr[RB], m[RB], d[RB], yy[RB];
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    kk[j] = Elem<Tin>::to_f(K[j * 32]);
+    vv[j] = Elem<Tin>::to_f(V[j * 32]);
+    rr[j] = GATE ? Elem<Tin>::to_f(R[j * 32]) : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j) m[j] = fmaf(float(j + 1), cp.w2, fmaf(kk[j], kLog2e, -s.pl));
+  float Q = s.Q;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) {
+    d[j] = m[j] - Q;
+    Q = fmaxf(Q, m[j]);
+  }
+  s.Q = Q;
+#pragma unroll
+  for (int j = 0; j < RB; ++j) yy[j] = wkv_token_d<GATE, FASTOUT>(s, cp, d[j], vv[j], rr[j]);
+#pragma unroll
+  for (int j = 0; j < RB; ++j) Y[j * 32] = Elem<Tin>::from_f(yy[j]);
+  wkv_rebase(s, float(RB) * cp.w2);
+}
+
 // Process n tokens of a tile already in shared memory (rows of 32 elements, this lane's
-// column), in windows of RB tokens. FULL: n == TT, fully unrolled; otherwise the window
-// length is the runtime value rb.
+// column). FULL: n == TT, in unrolled windows of RB tokens; otherwise token by token with
+// the runtime window length rb.
 template <typename Tin, bool GATE, bool FASTOUT, int TT, int RB, bool FULL>
 __device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, const Tin* K,
                                             const Tin* V, const Tin* R, Tin* Y, int n, int rb) {
   if (FULL) {
 #pragma unroll
-    for (int w0 = 0; w0 < TT; w0 += RB) {
-#pragma unroll
-      for (int j = 0; j < RB; ++j) {
-        const int row = (w0 + j) * 32;
-        const float k = Elem<Tin>::to_f(K[row]);
-        const float v = Elem<Tin>::to_f(V[row]);
-        const float r = GATE ? Elem<Tin>::to_f(R[row]) : 0.f;
-        Y[row] = Elem<Tin>::from_f(wkv_token<GATE, FASTOUT>(s, cp, float(j + 1), k, v, r));
-      }
-      wkv_rebase(s, float(RB) * cp.w2);
-    }
+    for (int w0 = 0; w0 < TT; w0 += RB)
+      window_tokens_smem<Tin, GATE, FASTOUT, RB>(s, cp, K + w0 * 32, V + w0 * 32, R + w0 * 32,
+                                                 Y + w0 * 32);
   } else {
     int j = 0;
     for (int t = 0; t < n; ++t) {

@@ -82,17 +82,15 @@ __device__ __forceinline__ float state_log_scale(const ChanState& s) {
   return fmaf(s.Q, kLn2, s.pl * kLn2);
 }
 
-// One token; fj = j as float (1-based position within the window).
+// One token given d = m_j - Q (its log2-weight against the state's running scale, with
+// Q already advanced by the caller): output and state update.
 template <bool GATE, bool FASTOUT>
-__device__ __forceinline__ float wkv_token(ChanState& s, const ChanParams& cp, float fj, float k,
-                                           float v, float r) {
-  const float m = fmaf(fj, cp.w2, fmaf(k, kLog2e, -s.pl));
-  const float d = m - s.Q;
+__device__ __forceinline__ float wkv_token_d(ChanState& s, const ChanParams& cp, float d, float v,
+                                             float r) {
   const float e = ex2(-fabsf(d));
   const bool c = d > 0.f;
   const float e1 = c ? e : 1.f;
   const float e2 = c ? 1.f : e;
-  s.Q = fmaxf(s.Q, m);
   float num, den;
   if (FASTOUT) {
     const float he = cp.H * e2;
@@ -117,6 +115,16 @@ __device__ __forceinline__ float wkv_token(ChanState& s, const ChanParams& cp, f
   s.a = fmaf(e1, s.a, e2 * v);
   s.b = fmaf(e1, s.b, e2);
   return num * rcp(den);
+}
+
+// One token; fj = j as float (1-based position within the window).
+template <bool GATE, bool FASTOUT>
+__device__ __forceinline__ float wkv_token(ChanState& s, const ChanParams& cp, float fj, float k,
+                                           float v, float r) {
+  const float m = fmaf(fj, cp.w2, fmaf(k, kLog2e, -s.pl));
+  const float d = m - s.Q;
+  s.Q = fmaxf(s.Q, m);
+  return wkv_token_d<GATE, FASTOUT>(s, cp, d, v, r);
 }
 
 // State update only (no output): used for chunk aggregates and recomputation.
