@@ -225,9 +225,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    Bn = args.batch
-    ELEMS = Bn * T * C
-    x = wkv_inputs.long_bf16(seed=rank, B=Bn)
+    Bn, Tn = args.batch, args.seq
+    ELEMS = Bn * Tn * C
+    x = wkv_inputs.long_bf16(seed=rank, B=Bn, T=Tn)
 
     def to_bf16(bits, pin=False):
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
@@ -314,7 +314,7 @@ def run_ours(args, rank, world, local_rank):
     if world == 1 and not args.no_cpu_baseline:
         rate, rows = cpu_oracle_rate(x, budget_s=10.0)
         cpu = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{rows} of {Bn} batch rows ({rows} x 4096 x 4096 elements) of the "
+               "sample": f"{rows} of {Bn} batch rows ({rows} x {Tn} x 4096 elements) of the "
                          f"same inputs, fp64 recurrence, 1 thread"}
     clocks = sampler.summary()
     out = {
@@ -322,11 +322,12 @@ def run_ours(args, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": f"WKV forward bf16 in/out, B={Bn} T=4096 C=4096 (7B-shaped, "
+        "config": {"workload": f"WKV forward bf16 in/out, B={Bn} T={Tn} C=4096 (7B-shaped, "
                                "k spikes of +60), one batch per GPU",
-                   "B": Bn, "T": T, "C": C, "storage": "bf16", "global_batch": Bn * world,
-                   "seq_len": T, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "inputs 805 MB + output 268 MB per step > 126 MB L2; no flush",
+                   "B": Bn, "T": Tn, "C": C, "storage": "bf16", "global_batch": Bn * world,
+                   "seq_len": Tn, "parallelism": f"dp{world} (independent batches)",
+                   "l2": f"inputs {3 * ELEMS * 2 / 1e6:.0f} MB + output {ELEMS * 2 / 1e6:.0f} MB "
+                         "per step > 126 MB L2; no flush",
                    "kernel": KERNEL},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": measured_traffic(),
@@ -353,6 +354,9 @@ def main():
     ap.add_argument("--batch", type=int, default=B,
                     help="batch rows per GPU (default 8, the measured workload; smaller "
                          "values are for profiler captures)")
+    ap.add_argument("--seq", type=int, default=T,
+                    help="tokens per sequence (default 4096, the measured workload; shorter "
+                         "sequences keep the occupancy of the full case for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -1,11 +1,13 @@
 // WKV forward over full sequences, one thread per (b, c) channel (sm_100a).
 //
-// Streaming kernel: one warp per CTA owns 32 adjacent channels of one batch row and walks
-// the whole sequence. Tiles of [TT tokens x 32 channels] of k, v, r are brought into
-// shared memory by TMA (3-D tensor maps over (C, T, B), so ragged T and C edges are
-// zero-filled on load and clipped on store), S stages deep, each stage on its own
-// mbarrier. y is staged in shared memory and written back by TMA store. The channel
-// state (a, b, P) lives in registers for the whole sequence.
+// Streaming kernel: a CTA of NW warps owns 32*NW adjacent channels of one batch row and
+// walks the whole sequence; each thread carries one channel's state (a, b, P) in registers.
+// Tiles of [TT tokens x 32*NW channels] of k, v, r are brought into shared memory by TMA
+// (3-D tensor maps over (C, T, B), so ragged T and C edges are zero-filled on load and
+// clipped on store), S stages deep, each stage on its own mbarrier; y is staged in shared
+// memory and written back by TMA store. For bf16 a CTA is two warps, so that every row of a
+// TMA box is 128 bytes: with 64-byte rows (one warp) the same streams reach about 15% less
+// DRAM bandwidth on B200 (measured with a compute-free probe of this access pattern).
 //
 // A plain kernel (direct coalesced global loads, same arithmetic) serves shapes the TMA
 // path cannot describe: C not a multiple of 4 (fp32) / 8 (bf16), or base pointers that
@@ -17,22 +19,21 @@
 
 namespace wkv {
 
-// One full window of RB tokens from shared memory, written in phases so that the only
-// serial chains are the ones the recurrence has (a running max for the scale, one fma per
-// token for a and b): every load of the window first, then the log-weights and their
-// running max, then the per-token arithmetic, then every store. (Token by token, each
-// token's loads would wait for the previous token's store, which the compiler must assume
-// may alias them.)
-template <typename Tin, bool GATE, bool FASTOUT, int RB>
-__device__ __forceinline__ void window_tokens_smem(ChanState& s, const ChanParams& cp,
-                                                   const Tin* K, const Tin* V, const Tin* R,
-                                                   Tin* Y) {
+// One full window of RB tokens from shared memory (row stride RS elements, this thread's
+// column), written in phases so that the only serial chains are the ones the recurrence
+// has (a running max for the scale, one fma per token for a and b): every load of the
+// window first, then the log-weights and their running max, then the per-token
+// arithmetic, then every store. (Token by token, each token's loads would wait for the
+// previous token's store, which the compiler must assume may alias them.)
+template <typename Tin, bool GATE, bool FASTOUT, int RB, int RS>
+__device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, const Tin* K,
+                                            const Tin* V, const Tin* R, Tin* Y) {
   float kk[RB], vv[RB], rr[RB], m[RB], d[RB], yy[RB];
 #pragma unroll
   for (int j = 0; j < RB; ++j) {
-    kk[j] = Elem<Tin>::to_f(K[j * 32]);
-    vv[j] = Elem<Tin>::to_f(V[j * 32]);
-    rr[j] = GATE ? Elem<Tin>::to_f(R[j * 32]) : 0.f;
+    kk[j] = Elem<Tin>::to_f(K[j * RS]);
+    vv[j] = Elem<Tin>::to_f(V[j * RS]);
+    rr[j] = GATE ? Elem<Tin>::to_f(R[j * RS]) : 0.f;
   }
 #pragma unroll
   for (int j = 0; j < RB; ++j) m[j] = fmaf(float(j + 1), cp.w2, fmaf(kk[j], kLog2e, -s.pl));
@@ -46,25 +47,25 @@ __device__ __forceinline__ void window_tokens_smem(ChanState& s, const ChanParam
 #pragma unroll
   for (int j = 0; j < RB; ++j) yy[j] = wkv_token_d<GATE, FASTOUT>(s, cp, d[j], vv[j], rr[j]);
 #pragma unroll
-  for (int j = 0; j < RB; ++j) Y[j * 32] = Elem<Tin>::from_f(yy[j]);
+  for (int j = 0; j < RB; ++j) Y[j * RS] = Elem<Tin>::from_f(yy[j]);
   wkv_rebase(s, float(RB) * cp.w2);
 }
 
-// Process n tokens of a tile already in shared memory (rows of 32 elements, this lane's
-// column). FULL: n == TT, in unrolled windows of RB tokens; otherwise token by token with
-// the runtime window length rb.
-template <typename Tin, bool GATE, bool FASTOUT, int TT, int RB, bool FULL>
+// Process n tokens of a tile in shared memory (row stride RS, this thread's column).
+// FULL: n == TT, in unrolled windows of RB tokens; otherwise token by token with the
+// runtime window length rb (the last, partial tile of a sequence).
+template <typename Tin, bool GATE, bool FASTOUT, int TT, int RB, int RS, bool FULL>
 __device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, const Tin* K,
                                             const Tin* V, const Tin* R, Tin* Y, int n, int rb) {
   if (FULL) {
 #pragma unroll
     for (int w0 = 0; w0 < TT; w0 += RB)
-      window_tokens_smem<Tin, GATE, FASTOUT, RB>(s, cp, K + w0 * 32, V + w0 * 32, R + w0 * 32,
-                                                 Y + w0 * 32);
+      window_smem<Tin, GATE, FASTOUT, RB, RS>(s, cp, K + w0 * RS, V + w0 * RS, R + w0 * RS,
+                                              Y + w0 * RS);
   } else {
     int j = 0;
     for (int t = 0; t < n; ++t) {
-      const int row = t * 32;
+      const int row = t * RS;
       const float k = Elem<Tin>::to_f(K[row]);
       const float v = Elem<Tin>::to_f(V[row]);
       const float r = GATE ? Elem<Tin>::to_f(R[row]) : 0.f;
@@ -78,30 +79,44 @@ __device__ __forceinline__ void tile_tokens(ChanState& s, const ChanParams& cp, 
   }
 }
 
-template <typename Tin, bool GATE, bool FASTOUT, int TT>
+template <typename Tin, bool GATE, bool FASTOUT, int TT, int RS>
 __device__ __forceinline__ void full_tile(ChanState& s, const ChanParams& cp, const Tin* K,
                                           const Tin* V, const Tin* R, Tin* Y, int rb) {
   if (rb == 16)
-    tile_tokens<Tin, GATE, FASTOUT, TT, 16, true>(s, cp, K, V, R, Y, TT, rb);
+    tile_tokens<Tin, GATE, FASTOUT, TT, 16, RS, true>(s, cp, K, V, R, Y, TT, rb);
   else if (rb == 4)
-    tile_tokens<Tin, GATE, FASTOUT, TT, 4, true>(s, cp, K, V, R, Y, TT, rb);
+    tile_tokens<Tin, GATE, FASTOUT, TT, 4, RS, true>(s, cp, K, V, R, Y, TT, rb);
   else
-    tile_tokens<Tin, GATE, FASTOUT, TT, 1, true>(s, cp, K, V, R, Y, TT, rb);
+    tile_tokens<Tin, GATE, FASTOUT, TT, 1, RS, true>(s, cp, K, V, R, Y, TT, rb);
 }
 
 // Largest window allowed for the output precision (see window_tokens).
 template <typename Tin>
-constexpr float window_limit() {
+__host__ __device__ constexpr float window_limit() {
   return sizeof(Tin) == 2 ? 512.f : 128.f;
 }
 
-template <typename Tin, bool GATE, int TT, int S>
-__global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
+__device__ __forceinline__ void cta_sync(int nw) {
+  if (nw == 1)
+    __syncwarp();
+  else
+    __syncthreads();
+}
+
+// Launch bounds: with no minimum, ptxas sizes registers for the 32-CTA residency limit
+// (32 registers at NW = 2), which serialises the windows; residency is bounded by shared
+// memory to a few CTAs per SM anyway, so ask for 4.
+template <typename Tin, bool GATE, int TT, int S, int NW>
+__global__ void __launch_bounds__(NW * 32, 4) wkv_fwd_tma_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_y, int T,
     int C, const float* __restrict__ w, const float* __restrict__ u, const float* a0,
     const float* b0, const float* p0, float* a1, float* b1, float* p1, unsigned* err) {
-  constexpr int kTile = TT * 32;
+  // Full tiles are processed in whole windows of up to 16 tokens.
+  static_assert(TT % 16 == 0, "tile length must be a multiple of the longest window");
+  static_assert(S >= 2, "the y staging wait below assumes two or more stages");
+  constexpr int CW = NW * 32;  // channels per CTA = elements per tile row
+  constexpr int kTile = TT * CW;
   constexpr uint32_t kTileBytes = kTile * sizeof(Tin);
   constexpr uint32_t kStageBytes = (GATE ? 3u : 2u) * kTileBytes;
 
@@ -112,23 +127,23 @@ __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
   Tin* sy = sr + (GATE ? S * kTile : 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sy + S * kTile);
 
-  const int lane = threadIdx.x;
-  const int G = (C + 31) >> 5;
+  const int tid = threadIdx.x;
+  const int G = (C + CW - 1) / CW;
   const int b = blockIdx.x / G;
   const int g = blockIdx.x - b * G;
-  const int c = (g << 5) + lane;
+  const int c = g * CW + tid;
   const bool valid = c < C;
   const int ntiles = (T + TT - 1) / TT;
 
   auto issue = [&](int stage, int tile) {
     uint64_t* bar = &bars[stage];
     mbar_arrive_expect_tx(bar, kStageBytes);
-    tma_load_3d(sk + stage * kTile, &tm_k, bar, g << 5, tile * TT, b);
-    tma_load_3d(sv + stage * kTile, &tm_v, bar, g << 5, tile * TT, b);
-    if (GATE) tma_load_3d(sr + stage * kTile, &tm_r, bar, g << 5, tile * TT, b);
+    tma_load_3d(sk + stage * kTile, &tm_k, bar, g * CW, tile * TT, b);
+    tma_load_3d(sv + stage * kTile, &tm_v, bar, g * CW, tile * TT, b);
+    if (GATE) tma_load_3d(sr + stage * kTile, &tm_r, bar, g * CW, tile * TT, b);
   };
 
-  if (lane == 0) {
+  if (tid == 0) {
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     if (GATE) prefetch_tmap(&tm_r);
@@ -138,45 +153,47 @@ __global__ void __launch_bounds__(32) wkv_fwd_tma_kernel(
     mbar_fence_init();
     for (int st = 0; st < S && st < ntiles; ++st) issue(st, st);
   }
-  __syncwarp();
+  cta_sync(NW);
 
   const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
   const size_t sidx = size_t(b) * C + c;
   const bool has_state = a0 != nullptr;
   ChanState s = (has_state && valid) ? load_state(a0[sidx], b0[sidx], p0[sidx]) : empty_state();
+  // Per-warp choices (window length, output form): warps of a CTA may differ.
   const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
   const int rb = window_tokens(cp.w2, window_limit<Tin>());
 
   for (int i = 0; i < ntiles; ++i) {
     const int st = i % S;
     mbar_wait(&bars[st], (i / S) & 1, err);
-    if (lane == 0 && i >= S) tma_store_wait_read<S - 1>();
-    __syncwarp();
-    const Tin* K = sk + st * kTile + lane;
-    const Tin* V = sv + st * kTile + lane;
-    const Tin* R = sr + st * kTile + lane;
-    Tin* Y = sy + st * kTile + lane;
+    const Tin* K = sk + st * kTile + tid;
+    const Tin* V = sv + st * kTile + tid;
+    const Tin* R = sr + st * kTile + tid;
+    Tin* Y = sy + st * kTile + tid;
     const int n = min(TT, T - i * TT);
     if (n == TT) {
       if (fast)
-        full_tile<Tin, GATE, true, TT>(s, cp, K, V, R, Y, rb);
+        full_tile<Tin, GATE, true, TT, CW>(s, cp, K, V, R, Y, rb);
       else
-        full_tile<Tin, GATE, false, TT>(s, cp, K, V, R, Y, rb);
+        full_tile<Tin, GATE, false, TT, CW>(s, cp, K, V, R, Y, rb);
     } else {
       if (fast)
-        tile_tokens<Tin, GATE, true, TT, 1, false>(s, cp, K, V, R, Y, n, rb);
+        tile_tokens<Tin, GATE, true, TT, 1, CW, false>(s, cp, K, V, R, Y, n, rb);
       else
-        tile_tokens<Tin, GATE, false, TT, 1, false>(s, cp, K, V, R, Y, n, rb);
+        tile_tokens<Tin, GATE, false, TT, 1, CW, false>(s, cp, K, V, R, Y, n, rb);
     }
+    // The y stage written next (tile i+1) was last stored as group i+1-S: let at most S-2
+    // of the groups committed so far (through i-1) still be reading shared memory.
+    if (tid == 0) tma_store_wait_read<S - 2>();
     fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_3d(&tm_y, sy + st * kTile, g << 5, i * TT, b);
+    cta_sync(NW);  // all of tile i read and all of its y written
+    if (tid == 0) {
+      tma_store_3d(&tm_y, sy + st * kTile, g * CW, i * TT, b);
       tma_store_commit();
       if (i + S < ntiles) issue(st, i + S);
     }
   }
-  if (lane == 0) tma_store_wait_all();
+  if (tid == 0) tma_store_wait_all();
 
   if (a1 != nullptr && valid) {
     a1[sidx] = s.a;
@@ -230,37 +247,63 @@ __global__ void __launch_bounds__(128) wkv_fwd_plain_kernel(
 // ---------------------------------------------------------------------------------------
 namespace {
 
-constexpr int kTT = 32;   // tokens per tile
+// Tile shape of the streaming kernel per element type: TT tokens per tile, S stages,
+// NW warps per CTA (32*NW channels, TMA box rows of 32*NW elements). The defaults come
+// from sweeps on B200; the macros exist for such sweeps.
+#ifndef WKV_FWD_TT_BF16
+#define WKV_FWD_TT_BF16 32
+#endif
+#ifndef WKV_FWD_S_BF16
+#define WKV_FWD_S_BF16 3
+#endif
+#ifndef WKV_FWD_NW_BF16
+#define WKV_FWD_NW_BF16 2
+#endif
+#ifndef WKV_FWD_TT_F32
+#define WKV_FWD_TT_F32 32
+#endif
+#ifndef WKV_FWD_S_F32
+#define WKV_FWD_S_F32 3
+#endif
+#ifndef WKV_FWD_NW_F32
+#define WKV_FWD_NW_F32 1
+#endif
 
-template <typename Tin>
-constexpr int stages() {
-  return 3;
-}
+template <typename Tin> struct FwdCfg;
+template <> struct FwdCfg<__nv_bfloat16> {
+  static constexpr int TT = WKV_FWD_TT_BF16, S = WKV_FWD_S_BF16, NW = WKV_FWD_NW_BF16;
+};
+template <> struct FwdCfg<float> {
+  static constexpr int TT = WKV_FWD_TT_F32, S = WKV_FWD_S_F32, NW = WKV_FWD_NW_F32;
+};
 
 template <typename Tin, bool GATE>
 size_t tma_smem_bytes() {
-  return size_t(stages<Tin>()) * (GATE ? 4 : 3) * kTT * 32 * sizeof(Tin) +
-         stages<Tin>() * sizeof(uint64_t);
+  using F = FwdCfg<Tin>;
+  return size_t(F::S) * ((GATE ? 3 : 2) + 1) * F::TT * F::NW * 32 * sizeof(Tin) +
+         F::S * sizeof(uint64_t);
 }
 
 template <typename Tin, bool GATE>
 int launch_tma(const FwdArgs& a, cudaStream_t stream) {
+  using F = FwdCfg<Tin>;
+  constexpr int CW = F::NW * 32;
   CUtensorMap tk, tv, tr, ty;
   const CUtensorMapDataType dt =
       sizeof(Tin) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  int rc = encode_btc_map(&tk, a.k, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
-  if (!rc) rc = encode_btc_map(&tv, a.v, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
-  if (!rc) rc = encode_btc_map(&tr, GATE ? a.r : a.k, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
-  if (!rc) rc = encode_btc_map(&ty, a.y, dt, sizeof(Tin), a.B, a.T, a.C, 32, kTT);
+  int rc = encode_btc_map(&tk, a.k, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
+  if (!rc) rc = encode_btc_map(&tv, a.v, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
+  if (!rc) rc = encode_btc_map(&tr, GATE ? a.r : a.k, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
+  if (!rc) rc = encode_btc_map(&ty, a.y, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
   if (rc) return rc;
-  auto kern = wkv_fwd_tma_kernel<Tin, GATE, kTT, stages<Tin>()>;
+  auto kern = wkv_fwd_tma_kernel<Tin, GATE, F::TT, F::S, F::NW>;
   const size_t smem = tma_smem_bytes<Tin, GATE>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return WKV_ERR_CUDA;
-  const int64_t G = (a.C + 31) / 32;
+  const int64_t G = (a.C + CW - 1) / CW;
   const int64_t grid = a.B * G;
-  kern<<<unsigned(grid), 32, smem, stream>>>(tk, tv, tr, ty, int(a.T), int(a.C), a.w, a.u, a.a0,
+  kern<<<unsigned(grid), CW, smem, stream>>>(tk, tv, tr, ty, int(a.T), int(a.C), a.w, a.u, a.a0,
                                              a.b0, a.p0, a.a1, a.b1, a.p1, a.err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
