@@ -35,7 +35,7 @@ UNIT = "G(B·T·C)/s"
 B, T, C = 8, 4096, 4096
 BYTES_PER_ELEM = 8          # read k, v, r and write y, 2 bytes each
 FALLBACK_HBM_GBS = 6650.0
-KERNEL = "wkv_fwd_tma_kernel<bf16, gate>"
+KERNEL = "wkv_fwd_tma_kernel<bf16, gate=1, TT=32, S=3, NW=1>"
 KERNEL_SOURCES = ["rwkv_linear_attention_wkv_b200/csrc/wkv_fwd.cu",
                   "rwkv_linear_attention_wkv_b200/csrc/wkv_step.cuh",
                   "rwkv_linear_attention_wkv_b200/csrc/wkv_device.cuh"]

@@ -5,9 +5,11 @@
 // Tiles of [TT tokens x 32*NW channels] of k, v, r are brought into shared memory by TMA
 // (3-D tensor maps over (C, T, B), so ragged T and C edges are zero-filled on load and
 // clipped on store), S stages deep, each stage on its own mbarrier; y is staged in shared
-// memory and written back by TMA store. For bf16 a CTA is two warps, so that every row of a
-// TMA box is 128 bytes: with 64-byte rows (one warp) the same streams reach about 15% less
-// DRAM bandwidth on B200 (measured with a compute-free probe of this access pattern).
+// memory and written back by TMA store. A CTA is one warp by default: with two warps the
+// bf16 boxes get 128-byte rows, which a compute-free probe of this access pattern streams
+// about 15% faster on B200, but the kernel as a whole measured no faster (it is bound by
+// per-warp issue of the recurrence, not by DRAM efficiency), and one-warp CTAs balance
+// better over 148 SMs (1024 CTAs at the 8 x 4096 x 4096 shape: 6.9 per SM).
 //
 // A plain kernel (direct coalesced global loads, same arithmetic) serves shapes the TMA
 // path cannot describe: C not a multiple of 4 (fp32) / 8 (bf16), or base pointers that
@@ -28,12 +30,13 @@ namespace wkv {
 template <typename Tin, bool GATE, bool FASTOUT, int RB, int RS>
 __device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, const Tin* K,
                                             const Tin* V, const Tin* R, Tin* Y) {
-  float kk[RB], vv[RB], rr[RB], m[RB], d[RB], yy[RB];
+  float kk[RB], vv[RB], m[RB], d[RB], den[RB], num[RB];
+  float rr[GATE ? RB : 1];
 #pragma unroll
   for (int j = 0; j < RB; ++j) {
     kk[j] = Elem<Tin>::to_f(K[j * RS]);
     vv[j] = Elem<Tin>::to_f(V[j * RS]);
-    rr[j] = GATE ? Elem<Tin>::to_f(R[j * RS]) : 0.f;
+    if (GATE) rr[j] = Elem<Tin>::to_f(R[j * RS]);
   }
 #pragma unroll
   for (int j = 0; j < RB; ++j) m[j] = fmaf(float(j + 1), cp.w2, fmaf(kk[j], kLog2e, -s.pl));
@@ -44,10 +47,45 @@ __device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, 
     Q = fmaxf(Q, m[j]);
   }
   s.Q = Q;
+  if (FASTOUT) {
+    // Exponentials of the window first (they depend on the scale chain only), then the
+    // fma chains of a and b, then the reciprocals: the MUFU pipe is never waiting on the
+    // chains, and the chains never wait on a MUFU result issued late.
+    float e[RB];
 #pragma unroll
-  for (int j = 0; j < RB; ++j) yy[j] = wkv_token_d<GATE, FASTOUT>(s, cp, d[j], vv[j], rr[j]);
+    for (int j = 0; j < RB; ++j) e[j] = ex2(-fabsf(d[j]));
+    float er[GATE ? RB : 1];
+    if (GATE) {
 #pragma unroll
-  for (int j = 0; j < RB; ++j) Y[j * RS] = Elem<Tin>::from_f(yy[j]);
+      for (int j = 0; j < RB; ++j) er[j] = ex2(rr[j] * -kLog2e);
+    }
+    float a = s.a, b = s.b;
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      const bool c = d[j] > 0.f;
+      const float e1 = c ? e[j] : 1.f;
+      const float e2 = c ? 1.f : e[j];
+      const float he = cp.H * e2;
+      num[j] = fmaf(e1, a, he * vv[j]);
+      den[j] = fmaf(e1, b, he);
+      if (GATE) den[j] = fmaf(den[j], er[j], den[j]);
+      a = fmaf(e1, a, e2 * vv[j]);
+      b = fmaf(e1, b, e2);
+    }
+    s.a = a;
+    s.b = b;
+  } else {
+#pragma unroll
+    for (int j = 0; j < RB; ++j) {
+      // generic output form, token by token; the returned value is num/den, folded below
+      const float y = wkv_token_d<GATE, false>(s, cp, d[j], vv[j], GATE ? rr[j] : 0.f);
+      num[j] = y;
+      den[j] = 1.f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < RB; ++j)
+    Y[j * RS] = Elem<Tin>::from_f(FASTOUT ? num[j] * rcp(den[j]) : num[j]);
   wkv_rebase(s, float(RB) * cp.w2);
 }
 
@@ -257,7 +295,7 @@ namespace {
 #define WKV_FWD_S_BF16 3
 #endif
 #ifndef WKV_FWD_NW_BF16
-#define WKV_FWD_NW_BF16 2
+#define WKV_FWD_NW_BF16 1
 #endif
 #ifndef WKV_FWD_TT_F32
 #define WKV_FWD_TT_F32 32

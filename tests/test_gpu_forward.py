@@ -81,6 +81,26 @@ def test_ragged_shapes_bf16(W, shape):
     assert_bf16_close(host_bf16(y), ref)
 
 
+@pytest.mark.parametrize("shape", [(2, 500, 192), (1, 4096, 64), (3, 65, 520)])
+def test_bf16_streaming_kernel_matches_plain_kernel_bitwise(W, shape):
+    # The TMA streaming kernel performs the same float operations as the plain kernel (only
+    # the data movement differs), so with equal window lengths the bits agree.
+    import ctypes
+    B, T, C = shape
+    x = wkv_inputs.make_inputs(B, T, C, seed=C + T, dtype="bf16", logw_range=(-6, 2),
+                               u_bound=2.0, k_std=3.0, spike_frac=1e-3)
+    w, u = dev(x.w), dev(x.u)
+    k, v, r = (dev_bf16(x.bits[n]) for n in "kvr")
+    y1 = W.wkv_forward_bf16(w, u, k, v, r)
+    y2 = torch.empty_like(y1)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    rc = W.lib.wkv_testing_forward_plain(B, T, C, P(w), P(u), P(k), P(v), P(r), P(y2), 1,
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    assert W.wkv_stream_status() == 0
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
 def test_single_token_is_v_and_constant_v(W):
     x = wkv_inputs.make_inputs(3, 1, 64, seed=3, k_std=5.0)
     y = run_f32(W, x, gate=False)
