@@ -61,7 +61,9 @@ typedef enum wkv_status {
   WKV_ERR_ALIGNMENT = 2,   /* a pointer not aligned to its element size                */
   WKV_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed              */
   WKV_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (wkv_stream_status)   */
-  WKV_ERR_UNSUPPORTED = 5  /* a size beyond what the kernels index (e.g. T >= 2^31)    */
+  WKV_ERR_UNSUPPORTED = 5, /* a size beyond what the kernels index (e.g. T >= 2^31)    */
+  WKV_ERR_SCRATCH_LIMIT = 6 /* wkv_forward_state_static: the problem needs more scratch
+                               than the library's fixed array holds                       */
 } wkv_status;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -110,6 +112,34 @@ WKV_API int wkv_forward_state(int64_t B, int64_t T, int64_t C, const float* w, c
                               const float* k, const float* v, const float* r, float* y,
                               const float* a0, const float* b0, const float* p0, float* a1,
                               float* b1, float* p1, cudaStream_t stream);
+
+/*
+ * wkv_forward_state without any device allocation. No counterpart in the pages: this is a
+ * deployment variant of the entry point above, for callers that cannot allocate device
+ * memory when they run the operator (a serving loop that must not risk the implicit
+ * device synchronisation an allocation can bring, a memory manager that owns all device
+ * memory, a deployment that forbids dynamic allocation after start-up).
+ *
+ * Same arguments, layout, semantics and results as wkv_forward_state; the caller passes
+ * all inputs and outputs. The scratch of the chunked path (look-back flags and carries,
+ * about 1 KiB per batch row x 32-channel group x 256-token segment) comes from a fixed
+ * array of 8 MiB in the library's device memory, which every GPU that loads the library
+ * holds until the process exits. Problems whose chunked
+ * plan needs more return WKV_ERR_SCRATCH_LIMIT before anything is enqueued; problems that
+ * take the streaming path need no scratch and have no limit. Nothing is allocated: no
+ * cudaMalloc, cudaMallocAsync or cudaFree (the flags are cleared with cudaMemsetAsync).
+ *
+ * The first call made with a given device current looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ * Every call shares the one array and leaves its contents behind: calls whose work
+ * overlaps on the GPU (different streams, or host threads not ordered with each other)
+ * race on it and give undefined results; order such calls, e.g. on one stream.
+ */
+WKV_API int wkv_forward_state_static(int64_t B, int64_t T, int64_t C, const float* w,
+                                     const float* u, const float* k, const float* v,
+                                     const float* r, float* y, const float* a0,
+                                     const float* b0, const float* p0, float* a1, float* b1,
+                                     float* p1, cudaStream_t stream);
 
 /*
  * One token for N sequences x L layers (recurrent inference; paper notes "关键设计 4",

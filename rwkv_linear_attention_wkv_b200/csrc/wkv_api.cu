@@ -72,6 +72,8 @@ int check_fwd(int64_t B, int64_t T, int64_t C, const void* w, const void* u, con
 
 }  // namespace
 
+unsigned* device_error_word() { return error_word(); }
+
 int encode_btc_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                    int elem_bytes, int64_t B, int64_t T, int64_t C, int box_c, int box_t) {
   auto enc = tensor_map_encoder();
@@ -165,6 +167,7 @@ WKV_API const char* wkv_status_string(int status) {
     case WKV_ERR_CUDA: return "WKV_ERR_CUDA";
     case WKV_ERR_TIMEOUT: return "WKV_ERR_TIMEOUT";
     case WKV_ERR_UNSUPPORTED: return "WKV_ERR_UNSUPPORTED";
+    case WKV_ERR_SCRATCH_LIMIT: return "WKV_ERR_SCRATCH_LIMIT";
     default: return "WKV_ERR_UNKNOWN";
   }
 }

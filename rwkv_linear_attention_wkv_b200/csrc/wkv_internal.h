@@ -30,6 +30,9 @@ struct FwdArgs {
   unsigned* err;  // device error word
 };
 
+// Device address of this library's error word on the current device (nullptr on error).
+unsigned* device_error_word();
+
 // 3-D tiled tensor map over a (B, T, C) tensor (C fastest) with a box of
 // [box_c channels x box_t tokens x 1 batch row]. Returns a wkv_status.
 int encode_btc_map(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
