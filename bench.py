@@ -138,6 +138,22 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise maximum of a list of floats over all ranks (identity without dist)."""
+    if dist is None:
+        return [float(x) for x in values]
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def aggregate_rate(world, elems_per_rank, steps, elapsed_ms):
+    """Whole-job throughput in G elements per second: every rank processed its own batch
+    `steps` times; the job took the slowest rank's time."""
+    return world * elems_per_rank * steps / (elapsed_ms / 1e3) / 1e9
+
+
 def visible_gpu_indices(n):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     if vis:
@@ -265,14 +281,9 @@ def run_ours(args, rank, world, local_rank):
     if W.wkv_stream_status() != 0:
         raise RuntimeError("device-side error during the timed region")
     per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    elapsed_ms = starts[0].elapsed_time(ends[-1])
-    if dist is not None:
-        t = torch.tensor([elapsed_ms, statistics.mean(per_launch)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, launch_ms = float(t[0]), float(t[1])
-    else:
-        launch_ms = statistics.mean(per_launch)
-    value = world * ELEMS * args.steps / (elapsed_ms / 1e3) / 1e9
+    elapsed_ms, launch_ms = max_over_ranks(
+        [starts[0].elapsed_time(ends[-1]), statistics.mean(per_launch)], dist, dev)
+    value = aggregate_rate(world, ELEMS, args.steps, elapsed_ms)
 
     # End to end through the public API: pinned host k, v, r -> device, forward, y -> host.
     e2e_steps = max(3, min(args.steps, 20))
@@ -297,12 +308,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t[0])
-    e2e_value = world * ELEMS * e2e_steps / (e2e_ms / 1e3) / 1e9
+    (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
+    e2e_value = aggregate_rate(world, ELEMS, e2e_steps, e2e_ms)
     assert np.array_equal(hy.view(torch.int16).numpy(), y.view(torch.int16).cpu().numpy()), \
         "end-to-end result differs from the device-resident run"
 
@@ -344,6 +351,90 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(out), flush=True)
 
 
+def _time_loop(fn, steps, warmup, stream):
+    """Mean milliseconds per call of fn over `steps` calls after `warmup` (CUDA events)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_workload(args):
+    """The other workloads the operator is checked on, measured on one GPU (one JSON line
+    each; the headline line above is the bf16 forward)."""
+    import numpy as np
+    import torch
+
+    import rwkv_linear_attention_wkv_b200 as W
+    import wkv_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peak, peak_kind = hbm_peak()
+
+    def d(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    def line(name, work, ms, elems, algo_bytes, extra=None):
+        gbs = algo_bytes / (ms / 1e3) / 1e9
+        out = {"workload": name, "work": work, "ms": ms,
+               "G_elem_per_s": elems / (ms / 1e3) / 1e9, "algorithmic_bytes": algo_bytes,
+               "achieved_GBps": gbs, "hbm_peak_GBps": peak, "peak_kind": peak_kind,
+               "frac": gbs / peak}
+        out.update(extra or {})
+        print(json.dumps(out), flush=True)
+
+    if args.workload == "train_169m":
+        x = wkv_inputs.training_shape(seed=0)
+        w, u, k, v, r, dy = (d(a) for a in (x.w, x.u, x.k, x.v, x.r, x.dy))
+        n = x.B * x.T * x.C
+        y = torch.empty_like(k)
+        ms = _time_loop(lambda: W.wkv_forward(w, u, k, v, r, y=y), args.steps, args.warmup, stream)
+        line("train_169m", "forward fp32 16x1024x768 (chunked kernel)", ms, n, 16 * n)
+        ws = torch.empty(W.wkv_backward_workspace_bytes(x.B, x.T, x.C), dtype=torch.uint8,
+                         device=dev)
+        out = {nm: torch.empty_like(k) for nm in ("dk", "dv", "dr")}
+        out["dw"] = torch.empty(x.C, device=dev)
+        out["du"] = torch.empty(x.C, device=dev)
+        ms = _time_loop(lambda: W.wkv_backward(w, u, k, v, r, dy, workspace=ws, out=out),
+                        args.steps, args.warmup, stream)
+        line("train_169m", "backward fp32 16x1024x768 (dk, dv, dr, dw, du)", ms, n, 28 * n)
+    elif args.workload == "long_ctx":
+        x = wkv_inputs.long_context(seed=0)
+        w, u, k, v, r = (d(a) for a in (x.w, x.u, x.k, x.v, x.r))
+        n = x.B * x.T * x.C
+        y = torch.empty_like(k)
+        st = tuple(torch.empty((x.B, x.C), device=dev) for _ in range(3))
+        ms = _time_loop(lambda: W.wkv_forward_state(w, u, k, v, r, y=y, state_out=st),
+                        args.steps, args.warmup, stream)
+        line("long_ctx", "forward_state fp32 1x32768x4096 (chunked kernel, final state)", ms, n,
+             16 * n + 12 * x.B * x.C)
+    elif args.workload == "decode":
+        dd = wkv_inputs.decode_batch(seed=0)
+        n = dd.N * dd.L * dd.C
+        w, u = d(dd.w), d(dd.u)
+        a, b, p = d(dd.a), d(dd.b), d(dd.p)
+        k, v, r = (d(t) for t in dd.step(0))
+        y = torch.empty_like(k)
+        ms = _time_loop(lambda: W.wkv_decode_step(w, u, k, v, r, a, b, p, y=y), args.steps,
+                        args.warmup, stream)
+        line("decode", "decode step fp32 256 seq x 32 layers x 4096 (state in place)", ms, n,
+             40 * n, {"tokens_per_s": dd.N / (ms / 1e3)})
+    else:
+        raise SystemExit(f"unknown workload {args.workload}")
+    if W.wkv_stream_status() != 0:
+        raise RuntimeError("device-side error")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -354,6 +445,10 @@ def main():
     ap.add_argument("--batch", type=int, default=B,
                     help="batch rows per GPU (default 8, the measured workload; smaller "
                          "values are for profiler captures)")
+    ap.add_argument("--workload", default="bf16_7b",
+                    choices=["bf16_7b", "train_169m", "long_ctx", "decode"],
+                    help="bf16_7b (default) prints the benchmark line; the others print "
+                         "measurements of the other workloads, one GPU")
     ap.add_argument("--seq", type=int, default=T,
                     help="tokens per sequence (default 4096, the measured workload; shorter "
                          "sequences keep the occupancy of the full case for profiler captures)")
@@ -381,6 +476,8 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.workload != "bf16_7b":
+        run_workload(args)
     else:
         run_ours(args, rank, world, local_rank)
 
