@@ -241,7 +241,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
 
-    Bn, Tn = args.batch, args.seq
+    Bn, Tn = args.batch, args.seq or T
     ELEMS = Bn * Tn * C
     x = wkv_inputs.long_bf16(seed=rank, B=Bn, T=Tn)
 
@@ -409,14 +409,14 @@ def run_workload(args):
                         args.steps, args.warmup, stream)
         line("train_169m", "backward fp32 16x1024x768 (dk, dv, dr, dw, du)", ms, n, 28 * n)
     elif args.workload == "long_ctx":
-        x = wkv_inputs.long_context(seed=0)
+        x = wkv_inputs.long_context(seed=0, T=args.seq or 32768)
         w, u, k, v, r = (d(a) for a in (x.w, x.u, x.k, x.v, x.r))
         n = x.B * x.T * x.C
         y = torch.empty_like(k)
         st = tuple(torch.empty((x.B, x.C), device=dev) for _ in range(3))
         ms = _time_loop(lambda: W.wkv_forward_state(w, u, k, v, r, y=y, state_out=st),
                         args.steps, args.warmup, stream)
-        line("long_ctx", "forward_state fp32 1x32768x4096 (chunked kernel, final state)", ms, n,
+        line("long_ctx", f"forward_state fp32 1x{x.T}x4096 (chunked kernel, final state)", ms, n,
              16 * n + 12 * x.B * x.C)
     elif args.workload == "decode":
         dd = wkv_inputs.decode_batch(seed=0)
@@ -449,9 +449,10 @@ def main():
                     choices=["bf16_7b", "train_169m", "long_ctx", "decode"],
                     help="bf16_7b (default) prints the benchmark line; the others print "
                          "measurements of the other workloads, one GPU")
-    ap.add_argument("--seq", type=int, default=T,
-                    help="tokens per sequence (default 4096, the measured workload; shorter "
-                         "sequences keep the occupancy of the full case for profiler captures)")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="tokens per sequence (default: the workload's own, 4096 for the "
+                         "benchmark; shorter sequences keep the occupancy of the full case "
+                         "for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -149,10 +149,10 @@ def test_invalid_arguments_raise(W):
 
 
 def test_training_shape_forward(W):
-    # B*C = 12288 channels: the chunked (time-parallel) kernel.
+    # B*C = 12288 channels: the streaming kernel (the plain kernel for comparison).
     x = wkv_inputs.training_shape(seed=0)
     ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r)
-    assert_fp32_close(run_f32(W, x), ref, "y (chunked)")
+    assert_fp32_close(run_f32(W, x), ref, "y (streaming)")
     assert_fp32_close(run_f32(W, x, plain=True), ref, "y (plain)")
     for b, c in wkv_inputs.sample_channels(x.B, x.C, 4):
         yd = oracle.wkv_direct(x.w[c:c + 1], x.u[c:c + 1], x.k[b:b + 1, :, c:c + 1],
