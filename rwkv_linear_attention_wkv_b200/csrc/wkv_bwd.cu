@@ -27,13 +27,17 @@
 //
 // Two kernels plus a reduction:
 //   1. checkpoint: one warp per 32 channels streams k, v forward (TMA) and stores the
-//      state entering every chunk of TT tokens;
-//   2. reverse: one warp per 32 channels walks the chunks from last to first; for each it
-//      loads k, v, r, dy, recomputes the forward factors from the chunk's checkpoint into
-//      shared memory, then runs the reverse recurrences and writes dk, dv (dr) in place of
-//      k, v (r) in shared memory for TMA stores; per-(b, c) partial sums of dw, du go to
-//      the workspace;
-//   3. reduce: dw[c], du[c] = sums over b in a fixed order (deterministic).
+//      state entering every chunk of kTT tokens;
+//   2. reverse, time-parallel (TMA shapes): one warp per chunk recomputes the chunk's
+//      forward from its checkpoint, the carries of the reverse sums are chained across
+//      segments of kSW chunks, and each warp then runs the reverse over its chunk (see
+//      section 2' below). Shapes TMA cannot address take the serial form: one warp per 32
+//      channels walks the chunks from last to first, recomputing each chunk's factors into
+//      shared memory before its reverse;
+//   both write dk, dv (dr) in place of k, v (r) in shared memory for the stores, and
+//   per-(b, chunk, c) partial sums of dw, du to the workspace;
+//   3. reduce: dw[c], du[c] = sums of the per-chunk partials over b and t in a fixed order
+//      (deterministic).
 #include <algorithm>
 
 #include "wkv_internal.h"
@@ -43,31 +47,73 @@ namespace wkv {
 
 namespace {
 
-constexpr int kTT = 32;  // tokens per chunk
+constexpr int kTT = 16;   // tokens per chunk (checkpoint interval; one warp's unit of work)
+constexpr int kSW = 4;    // chunks (warps) per segment of the time-parallel passes
+// Segments whose results a segment folds in directly before taking a carry from further
+// away (which makes one link of a serial chain per kFoldF / kFoldR + 1 segments): in the
+// checkpoint pass (forward) and the reverse pass.
+constexpr int kFoldF = 16;
+constexpr int kFoldR = 5;
 
 struct BwdLayout {
-  float4* ckpt;  // [B, nchunks, C] state entering each chunk: (a, b, Q, pl)
-  float* pdw;    // [B, C]
-  float* pdu;    // [B, C]
+  float4* ckpt;      // [B, nch, C] forward state entering each chunk: (a, b, Q, pl)
+  float* pdw;        // [B, nseg, C] per-segment partial sums of dw
+  float* pdu;        // [B, nseg, C] per-segment partial sums of du
+  unsigned* fticket;  // segment tickets of the checkpoint pass (forward chain)
+  unsigned* rticket;  // segment tickets of the reverse pass (reverse chain)
+  unsigned* fflags;   // [nbg * nseg]: 1 once the segment's aggregate is published, 2 once the
+                      // state entering it (its first checkpoint) is written
+  unsigned* rflags;   // [nbg * nseg]: 1 once the segment's reverse map is published, 2 its carry
+  float4* fagg;      // [nbg * nseg, 32]: the segment's forward aggregate (a, b, ph, pl)
+  float4* rmap;      // [nbg * nseg, 32, 2]: the segment's reverse map (see RevAgg)
+  float4* carry;     // [nbg * nseg, 32]: (beta, gamma, betad, gammad) at the segment start
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+__host__ __device__ inline int64_t bwd_nseg(int64_t T) {
+  const int64_t nch = (T + kTT - 1) / kTT;
+  return (nch + kSW - 1) / kSW;
+}
+
+// Bytes of the chain flags (with the tickets) that must be zero at the start of a call.
+__host__ __device__ inline size_t bwd_flag_bytes(int64_t B, int64_t T, int64_t C) {
+  const int64_t nitems = B * ((C + 31) / 32) * bwd_nseg(T);
+  return align256(size_t(16 + 8 * nitems));
+}
+
 __host__ __device__ inline BwdLayout bwd_layout(void* ws, int64_t B, int64_t T, int64_t C) {
   const int64_t nch = (T + kTT - 1) / kTT;
+  const int64_t nitems = B * ((C + 31) / 32) * bwd_nseg(T);
   char* p = static_cast<char*>(ws);
   BwdLayout L;
+  L.fticket = reinterpret_cast<unsigned*>(p);
+  L.rticket = reinterpret_cast<unsigned*>(p + 4);
+  L.fflags = reinterpret_cast<unsigned*>(p + 16);
+  L.rflags = L.fflags + nitems;
+  p += bwd_flag_bytes(B, T, C);
   L.ckpt = reinterpret_cast<float4*>(p);
   p += align256(size_t(B) * nch * C * sizeof(float4));
   L.pdw = reinterpret_cast<float*>(p);
-  p += align256(size_t(B) * C * sizeof(float));
+  p += align256(size_t(B) * bwd_nseg(T) * C * sizeof(float));
   L.pdu = reinterpret_cast<float*>(p);
+  p += align256(size_t(B) * bwd_nseg(T) * C * sizeof(float));
+  L.fagg = reinterpret_cast<float4*>(p);
+  p += align256(size_t(nitems) * 32 * sizeof(float4));
+  L.rmap = reinterpret_cast<float4*>(p);
+  p += align256(size_t(nitems) * 32 * 2 * sizeof(float4));
+  L.carry = reinterpret_cast<float4*>(p);
   return L;
 }
 
 __host__ __device__ inline size_t bwd_bytes(int64_t B, int64_t T, int64_t C) {
   const int64_t nch = (T + kTT - 1) / kTT;
-  return align256(size_t(B) * nch * C * sizeof(float4)) + 2 * align256(size_t(B) * C * sizeof(float));
+  const int64_t nitems = B * ((C + 31) / 32) * bwd_nseg(T);
+  return bwd_flag_bytes(B, T, C) + align256(size_t(B) * nch * C * sizeof(float4)) +
+         2 * align256(size_t(B) * bwd_nseg(T) * C * sizeof(float)) +
+         align256(size_t(nitems) * 32 * sizeof(float4)) +
+         align256(size_t(nitems) * 32 * 2 * sizeof(float4)) +
+         align256(size_t(nitems) * 32 * sizeof(float4));
 }
 
 // ---- tile movement: TMA, or plain per-lane loads/stores for unaligned shapes ----------
@@ -145,6 +191,11 @@ struct Tiles {
     if (TMA && lane == 0) tma_store_wait_all();
     __syncwarp();
   }
+  // Only until the stores have read their shared-memory sources (enough to refill them).
+  static __device__ __forceinline__ void store_read_drain(int lane) {
+    if (TMA && lane == 0) tma_store_wait_read<0>();
+    __syncwarp();
+  }
 };
 
 struct TensorMaps4 {
@@ -153,7 +204,7 @@ struct TensorMaps4 {
 
 // ---- 1. checkpoints --------------------------------------------------------------------
 template <bool TMA>
-__global__ void __launch_bounds__(32) wkv_bwd_ckpt_kernel(const __grid_constant__ TensorMaps4 maps,
+__global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_constant__ TensorMaps4 maps,
                                                           const float* __restrict__ k,
                                                           const float* __restrict__ v,
                                                           int B, int T, int C,
@@ -204,11 +255,177 @@ __global__ void __launch_bounds__(32) wkv_bwd_ckpt_kernel(const __grid_constant_
   }
 }
 
+// Token weights for the time-parallel checkpoints and the recomputation that starts from
+// them. The checkpoint after a chunk is its entering state combined with the chunk's own
+// aggregate (from the empty state), while the reverse pass recomputes the same chunk from the
+// entering state; the two must weigh every token identically, or a dominant token (a
+// spike in k) would carry two different roundings of its weight into the two sides and
+// the reverse sums would be inconsistent at the level of ulp(k log2 e). So the token's
+// log2-weight in the window, m = k log2(e) + j w2, is rounded independently of the state,
+// and the state's low part enters only the comparison d = (m - Q) - pl; a token that
+// takes over the scale sets it to (m, 0).
+// The product is rounded on its own (__fmul_rn): with fj a compile-time 1 the compiler
+// could otherwise fuse it into the fma, and the two kernels would round differently.
+__device__ __forceinline__ float tok_log2w(float fj, float w2, float k) {
+  return fmaf(fj, w2, __fmul_rn(k, kLog2e));
+}
+
+__device__ __forceinline__ void absorb_indep(ChanState& s, const ChanParams& cp, float fj, float k,
+                                             float v) {
+  const float m = tok_log2w(fj, cp.w2, k);
+  const float d = (m - s.Q) - s.pl;
+  const float e = ex2(-fabsf(d));
+  const bool c = d > 0.f;
+  const float e1 = c ? e : 1.f;
+  const float e2 = c ? 1.f : e;
+  s.Q = c ? m : s.Q;
+  s.pl = c ? 0.f : s.pl;
+  s.a = fmaf(e1, s.a, e2 * v);
+  s.b = fmaf(e1, s.b, e2);
+}
+
+// Time-parallel form (TMA shapes). One CTA per (segment of kSW chunks, batch row, 32-channel
+// group), warp i on chunk kSW seg + i; CTAs take segments in ticket order from the first on,
+// so every segment a CTA waits for belongs to a CTA that started earlier. Each warp folds its
+// chunk's k, v into the chunk's aggregate from the empty state. Before its own chunk, the
+// last warp forms the state entering the segment, in a fixed order (bitwise reproducible):
+// the state entering segment j0 = max(0, seg - kFoldF) (its first checkpoint), then the
+// published aggregates of segments j0 .. seg-1; so one link of a serial chain spans kFoldF
+// segments. After one barrier each warp combines that state with the aggregates of the
+// chunks before its own and writes its chunk's checkpoint; warp 0 publishes the segment's
+// aggregate. One pass, 8 bytes of HBM reads per element.
+__global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
+    const __grid_constant__ TensorMaps4 maps, int B, int T, int C, const float* __restrict__ w,
+    void* ws, unsigned* err) {
+  constexpr int kTile = kTT * 32;
+  __shared__ __align__(128) float tiles[kSW][2][kTile];  // k, v per warp
+  __shared__ float4 sagg[kSW][32];
+  __shared__ float4 sfold[kFoldF][32];  // earlier segments' aggregates
+  __shared__ float4 sin_[32];           // the state entering the segment
+  __shared__ uint64_t bars[kSW];
+  __shared__ unsigned s_ticket;
+
+  const int G = (C + 31) >> 5;
+  const int64_t nbg = int64_t(B) * G;
+  const int nch = (T + kTT - 1) / kTT;
+  const int nseg = (nch + kSW - 1) / kSW;
+  const BwdLayout lay = bwd_layout(ws, B, T, C);
+  if (threadIdx.x == 0) s_ticket = atomicAdd(lay.fticket, 1u);
+  __syncthreads();
+  const int64_t ticket = s_ticket;
+  const int seg = int(ticket / nbg);
+  const int64_t bg = ticket - int64_t(seg) * nbg;
+  const int b = int(bg / G);
+  const int g = int(bg - int64_t(b) * G);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = (g << 5) + lane;
+  const bool valid = c < C;
+  const int ch = seg * kSW + warp;
+  const int n = max(0, min(kTT, T - ch * kTT));  // tokens of this warp's chunk
+  const int64_t item0 = bg * nseg;
+  const int64_t item = item0 + seg;
+  float4* ck = lay.ckpt + int64_t(b) * nch * C + c;  // checkpoint of chunk i at ck[i * C]
+
+  uint64_t* bar = &bars[warp];
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+    if (n > 0) {
+      mbar_arrive_expect_tx(bar, 2u * kTile * sizeof(float));
+      tma_load_3d(&tiles[warp][0][0], &maps.m[0], bar, g << 5, ch * kTT, b);
+      tma_load_3d(&tiles[warp][1][0], &maps.m[1], bar, g << 5, ch * kTT, b);
+    }
+  }
+  __syncwarp();
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, 0.f);
+  const int rb = window_tokens(cp.w2, 128.f);
+
+  // ---- the chunk's aggregate from the empty state ----
+  Agg A = agg_empty();
+  if (n > 0) {
+    mbar_wait(bar, 0, err);
+    __syncwarp();
+    ChanState s = empty_state();
+    int j = 0;
+    for (int t = 0; t < n; ++t) {
+      absorb_indep(s, cp, float(j + 1), tiles[warp][0][t * 32 + lane], tiles[warp][1][t * 32 + lane]);
+      if (++j == rb) {
+        wkv_rebase(s, float(rb) * cp.w2);
+        j = 0;
+      }
+    }
+    if (j) wkv_rebase_partial(s, j, cp.w2);
+    A = to_agg(s);
+  }
+  sagg[warp][lane] = make_float4(A.a, A.b, A.ph, A.pl);
+  __syncthreads();
+
+  // ---- the segment's aggregate, for the segments after it ----
+  const bool first = seg > 0 && seg + kFoldF < nseg;  // segment seg + kFoldF starts here
+  if (warp == 0 && seg + 1 < nseg) {
+    Agg S = agg_empty();
+#pragma unroll
+    for (int i = 0; i < kSW; ++i) {
+      const float4 q = sagg[i][lane];
+      S = combine(S, Agg{q.x, q.y, q.z, q.w}, float(kTT), cp.w2);  // all chunks full
+    }
+    lay.fagg[item * 32 + lane] = make_float4(S.a, S.b, S.ph, S.pl);
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release(&lay.fflags[item], 1u);
+  }
+  // ---- the state entering the segment (last warp; the aggregate above does not wait) ----
+  if (warp == kSW - 1) {
+    const int j0 = max(0, seg - kFoldF);
+    const int m = seg - j0;  // aggregates to fold
+    unsigned fl = 1;
+    if (lane < m) fl = wait_flag(&lay.fflags[item0 + j0 + lane], 1u, kWaitLimitNs, err);
+    if (lane == 31 && j0 > 0) fl = wait_flag(&lay.fflags[item0 + j0], 2u, kWaitLimitNs, err);
+    const bool ok = __all_sync(0xffffffffu, fl != 0);
+    Agg X = agg_empty();
+    if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
+      // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
+      for (int l = 0; l < m; ++l) sfold[l][lane] = __ldcg(&lay.fagg[(item0 + j0 + l) * 32 + lane]);
+      if (j0 > 0 && valid) {
+        const float4 q = __ldcg(&ck[int64_t(j0) * kSW * C]);
+        X = Agg{q.x, q.y, q.z, q.w};
+      }
+      __syncwarp();
+      for (int l = 0; l < m; ++l) {
+        const float4 a = sfold[l][lane];
+        X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kSW * kTT), cp.w2);
+      }
+    }
+    sin_[lane] = make_float4(X.a, X.b, X.ph, X.pl);
+  }
+
+  __syncthreads();
+
+  // ---- checkpoints ----
+  {
+    const float4 q = sin_[lane];
+    Agg X{q.x, q.y, q.z, q.w};
+    for (int i = 0; i < warp; ++i) {  // chunks before this one (full)
+      const float4 a = sagg[i][lane];
+      X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kTT), cp.w2);
+    }
+    if (n > 0 && valid) ck[int64_t(ch) * C] = make_float4(X.a, X.b, X.ph, X.pl);
+  }
+  if (warp == 0 && first) {  // the first checkpoint is written: release it
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release(&lay.fflags[item], 2u);
+  }
+}
+
 // ---- 2. reverse pass ---------------------------------------------------------------------
-// Shared memory per CTA (floats): 2 stages x 4 tiles (k, v, r, dy; dk, dv, dr written in
+// Shared memory per CTA (floats): kMS stages x 4 tiles (k, v, r, dy; dk, dv, dr written in
 // place of k, v, r) + 6 factor tiles (e1, e2, f_inj, f_cur, wkv, sigma).
+constexpr int kMS = 3;
+// Launch bounds with a minimum of 3 resident CTAs (all that shared memory allows): without
+// one, ptxas budgets registers for 32 CTAs per SM (64 per thread).
 template <bool TMA, bool GATE, bool DR>
-__global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
+__global__ void __launch_bounds__(32, 3) wkv_bwd_main_kernel(
     const __grid_constant__ TensorMaps4 in_maps, const __grid_constant__ TensorMaps4 out_maps,
     const float* __restrict__ k, const float* __restrict__ v, const float* __restrict__ r,
     const float* __restrict__ dy, float* dk, float* dv, float* dr, int B, int T, int C,
@@ -216,7 +433,7 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
   constexpr int kTile = kTT * 32;
   extern __shared__ __align__(128) float smem[];
   // stage s2 holds tiles k, v, r (or dy), dy at smem + (4 s2 + slot) kTile
-  float* fe1 = smem + 8 * kTile;
+  float* fe1 = smem + 4 * kMS * kTile;
   float* fe2 = fe1 + kTile;
   float* finj = fe2 + kTile;
   float* fcur = finj + kTile;
@@ -242,8 +459,7 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
                      T, C, lane);
   };
   if (lane == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int st = 0; st < kMS; ++st) mbar_init(&bars[st], 1);
     mbar_fence_init();
   }
   __syncwarp();
@@ -255,12 +471,18 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
   float beta = 0.f, gamma = 0.f, betad = 0.f, gammad = 0.f;  // scaled suffix sums
   float dw_acc = 0.f, du_acc = 0.f;
 
-  issue(0, nch - 1);
-  if (nch > 1) issue(1, nch - 2);
+  for (int st = 0; st < kMS && st < nch; ++st) issue(st, nch - 1 - st);
+  auto ckpt_of = [&](int ch) {
+    return valid ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
+                 : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
+  };
+  float4 ck_next = ckpt_of(nch - 1);  // checkpoints are read one chunk ahead
   for (int it = 0; it < nch; ++it) {
     const int ch = nch - 1 - it;
-    const int s2 = it & 1;
-    Tiles<TMA>::wait(&bars[s2], (it >> 1) & 1, err);
+    const int s2 = it % kMS;
+    const float4 ck = ck_next;
+    if (ch > 0) ck_next = ckpt_of(ch - 1);
+    Tiles<TMA>::wait(&bars[s2], (it / kMS) & 1, err);
     float* K = smem + (4 * s2 + 0) * kTile;
     float* V = smem + (4 * s2 + 1) * kTile;
     float* R = smem + (4 * s2 + 2) * kTile;
@@ -268,14 +490,13 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
     const int n = min(kTT, T - ch * kTT);
 
     // Forward recomputation of the chunk from its checkpoint: per-token factors.
-    float4 ck = valid ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
-                      : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
     ChanState s;
     s.a = ck.x;
     s.b = ck.y;
     s.Q = ck.z;
     s.pl = ck.w;
     int j = 0;
+#pragma unroll 8
     for (int t = 0; t < n; ++t) {
       const int o = t * 32 + lane;
       const float kk = K[o], vv = V[o];
@@ -322,6 +543,7 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
       }
     }
     // Reverse over the chunk; dk, dv (dr) replace k, v (r) in shared memory.
+#pragma unroll 8
     for (int t = n - 1; t >= 0; --t) {
       const int o = t * 32 + lane;
       const float gy = DY[o], vv = V[o];
@@ -342,35 +564,435 @@ __global__ void __launch_bounds__(32) wkv_bwd_main_kernel(
       beta = fmaf(e1, beta, inj);
       gamma = fmaf(e1, gamma, inj * wk);
     }
+    if (ch % kSW == 0) {  // the segment's first chunk: its partial sums are complete
+      if (valid) {
+        const int64_t nseg = bwd_nseg(T);
+        lay.pdw[(int64_t(b) * nseg + ch / kSW) * C + c] = -dw_acc;
+        lay.pdu[(int64_t(b) * nseg + ch / kSW) * C + c] = du_acc;
+      }
+      dw_acc = 0.f;
+      du_acc = 0.f;
+    }
     Tiles<TMA>::store(out_maps.m, outp, nstore, K, b, g, ch * kTT, T, C, lane);
-    if (it + 2 < nch) {
-      // The stores read this stage's tiles: drain them before the refill overwrites.
-      Tiles<TMA>::store_drain(lane);
-      issue(s2, ch - 2);
+    if (it + kMS < nch) {
+      // The stores read this stage's tiles: let them finish reading before the refill.
+      Tiles<TMA>::store_read_drain(lane);
+      issue(s2, ch - kMS);
     }
   }
   Tiles<TMA>::store_drain(lane);
-  if (valid) {
-    lay.pdw[int64_t(b) * C + c] = -dw_acc;
-    lay.pdu[int64_t(b) * C + c] = du_acc;
-  }
 }
 
-// ---- 3. reduction over the batch, fixed order ----------------------------------------------
-__global__ void wkv_bwd_reduce_kernel(int B, int C, const void* ws, int T, float* dw, float* du) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= C) return;
+// ---- 2'. time-parallel reverse pass ------------------------------------------------------
+// The reverse recurrences are linear in the carried sums, so a span of L tokens acts on the
+// carry X = (beta~, gamma~, betad~, gammad~) at its end as an affine map: with E the product
+// of the forward factors e1 over the span and (lb, lg, lbd, lgd) the span's own sums from a
+// zero carry,
+//   beta' = E beta + lb,  gamma' = E gamma + lg,
+//   betad' = E (betad + L beta) + lbd,  gammad' = E (gammad + L gamma) + lgd
+// (unrolling betad_{i-1} = e1_i (betad_i + beta_i) over the span). The maps of the chunks
+// come out of the parallel forward recomputation; only the cheap application of a
+// segment's maps to its carry is serial, chained from the last segment to the first.
+struct RevAgg {
+  float E, L, lb, lg, lbd, lgd;
+};
+struct RevCarry {
+  float b, g, bd, gd;
+};
+
+__device__ __forceinline__ RevAgg rev_identity() { return RevAgg{1.f, 0.f, 0.f, 0.f, 0.f, 0.f}; }
+
+// The carry at the start of span A, given the carry X at its end.
+__device__ __forceinline__ RevCarry rev_apply(const RevAgg& A, const RevCarry& X) {
+  RevCarry r;
+  r.b = fmaf(A.E, X.b, A.lb);
+  r.g = fmaf(A.E, X.g, A.lg);
+  r.bd = fmaf(A.E, fmaf(A.L, X.b, X.bd), A.lbd);
+  r.gd = fmaf(A.E, fmaf(A.L, X.g, X.gd), A.lgd);
+  return r;
+}
+
+// A1 directly before A2 in time: rev_apply(rev_compose(A1, A2), X) = rev_apply(A1, rev_apply(A2, X)).
+__device__ __forceinline__ RevAgg rev_compose(const RevAgg& A1, const RevAgg& A2) {
+  RevAgg r;
+  r.E = A1.E * A2.E;
+  r.L = A1.L + A2.L;
+  r.lb = fmaf(A1.E, A2.lb, A1.lb);
+  r.lg = fmaf(A1.E, A2.lg, A1.lg);
+  r.lbd = fmaf(A1.E, fmaf(A1.L, A2.lb, A2.lbd), A1.lbd);
+  r.lgd = fmaf(A1.E, fmaf(A1.L, A2.lg, A2.lgd), A1.lgd);
+  return r;
+}
+
+__device__ __forceinline__ void put_agg(float4* p, const RevAgg& A) {
+  p[0] = make_float4(A.E, A.lb, A.lg, A.lbd);
+  p[1] = make_float4(A.lgd, A.L, 0.f, 0.f);
+}
+__device__ __forceinline__ RevAgg get_agg(float4 x, float4 y) {
+  return RevAgg{x.x, y.y, x.y, x.z, x.w, y.x};
+}
+
+// Per-token factors of one chunk from the forward recomputation, kept in registers (every
+// index is a compile-time constant after unrolling). e1/e2: one of them is 1, the other is
+// fe[t]; bit t of `tok` says which (set: the token's own term dominated, e1 = fe[t],
+// e2 = 1). inj and cur already carry the token's dy.
+struct ChunkFactors {
+  float fe[kTT], inj[kTT], cur[kTT], wkv[kTT];
+  unsigned tok;
+};
+
+// Forward recomputation of one chunk of kTT tokens from its entering state s (left holding
+// the state after the chunk): fills the per-token factors, writes dr in place of r (DR),
+// and returns the chunk's reverse map (its sums from a zero carry, composed token by token
+// in time order).
+template <bool GATE, bool DR, bool FASTOUT, int RB>
+__device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& cp, const float* K,
+                                                const float* V, float* R, const float* DY,
+                                                ChunkFactors& f) {
+  static_assert(kTT % RB == 0, "windows must tile the chunk");
+  RevAgg A = rev_identity();
+  f.tok = 0u;
+#pragma unroll
+  for (int t = 0; t < kTT; ++t) {
+    const float kk = K[t * 32], vv = V[t * 32], gy = DY[t * 32];
+    const float m = tok_log2w(float(t % RB + 1), cp.w2, kk);  // as absorb_indep
+    const float d = (m - s.Q) - s.pl;
+    const float e = ex2(-fabsf(d));
+    const bool cnd = d > 0.f;
+    const float e1 = cnd ? e : 1.f;
+    const float e2 = cnd ? 1.f : e;
+    s.Q = cnd ? m : s.Q;
+    s.pl = cnd ? 0.f : s.pl;
+    float num, den, ki, kc;
+    if (FASTOUT) {
+      const float he = cp.H * e2;
+      num = fmaf(e1, s.a, he * vv);
+      den = fmaf(e1, s.b, he);
+      ki = e1;
+      kc = he;
+    } else {
+      const float dO = d + cp.uw2;
+      const float oo = ex2(-fabsf(dO));
+      const bool co = dO > 0.f;
+      const float o1 = co ? oo : 1.f;
+      const float o2 = co ? 1.f : oo;
+      num = fmaf(o1, s.a, o2 * vv);
+      den = fmaf(o1, s.b, o2);
+      ki = o1;
+      kc = o2;
+    }
+    const float rden = rcp(den);
+    float sig = 1.f;
+    if (GATE) sig = rcp(1.f + ex2(R[t * 32] * -kLog2e));
+    const float h = gy * sig * rden;  // dy sigmoid(r) / den
+    const float wk = num * rden;
+    const float inj = h * ki;
+    f.fe[t] = e;
+    f.tok |= cnd ? (1u << t) : 0u;
+    f.inj[t] = inj;
+    f.cur[t] = h * kc;
+    f.wkv[t] = wk;
+    if (DR) R[t * 32] = gy * wk * sig * (1.f - sig);  // dr in place of r
+    // Compose the single-token map (E = e1, L = 1, l_beta = inj, l_gamma = inj wkv) after A.
+    const float ej = A.E * inj;
+    A.lbd = fmaf(ej, float(t), A.lbd);
+    A.lgd = fmaf(ej * wk, float(t), A.lgd);
+    A.lb += ej;
+    A.lg = fmaf(ej, wk, A.lg);
+    A.E *= e1;
+    s.a = fmaf(e1, s.a, e2 * vv);
+    s.b = fmaf(e1, s.b, e2);
+    if ((t + 1) % RB == 0) wkv_rebase(s, float(RB) * cp.w2);
+  }
+  A.L = float(kTT);
+  return A;
+}
+
+template <bool GATE, bool DR, bool FASTOUT>
+__device__ __forceinline__ RevAgg chunk_forward_rb(ChanState& s, const ChanParams& cp, int rb,
+                                                   const float* K, const float* V, float* R,
+                                                   const float* DY, ChunkFactors& f) {
+  if (rb == 16) return chunk_forward<GATE, DR, FASTOUT, 16>(s, cp, K, V, R, DY, f);
+  if (rb == 4) return chunk_forward<GATE, DR, FASTOUT, 4>(s, cp, K, V, R, DY, f);
+  return chunk_forward<GATE, DR, FASTOUT, 1>(s, cp, K, V, R, DY, f);
+}
+
+// Reverse over one chunk from the carry X at its end: dk, dv replace k, v in shared memory;
+// returns the chunk's partial sums of -dw (.x) and du (.y).
+__device__ __forceinline__ float2 chunk_reverse(const ChunkFactors& f, RevCarry X, float* K,
+                                                float* V) {
+  float dw_acc = 0.f, du_acc = 0.f;
+#pragma unroll
+  for (int t = kTT - 1; t >= 0; --t) {
+    const float vv = V[t * 32];
+    const bool dom = (f.tok >> t) & 1u;
+    const float e1 = dom ? f.fe[t] : 1.f;
+    const float e2 = dom ? 1.f : f.fe[t];
+    const float wk = f.wkv[t], inj = f.inj[t], cur = f.cur[t];
+    const float vm = vv - wk;
+    V[t * 32] = fmaf(e2, X.b, cur);                            // dv
+    K[t * 32] = fmaf(cur, vm, e2 * fmaf(vv, X.b, -X.g));       // dk
+    dw_acc = fmaf(e2, fmaf(vv, X.bd, -X.gd), dw_acc);
+    du_acc = fmaf(cur, vm, du_acc);
+    X.bd = e1 * (X.bd + X.b);
+    X.gd = e1 * (X.gd + X.g);
+    X.b = fmaf(e1, X.b, inj);
+    X.g = fmaf(e1, X.g, inj * wk);
+  }
+  return make_float2(-dw_acc, du_acc);
+}
+
+// Persistent CTAs of kSW warps; each takes segment items (a segment of kSW chunks of one
+// batch row and 32-channel group) in ticket order from the LAST segment backward, so every
+// segment an item waits for has a smaller ticket: it is done or in progress, and the
+// smallest item in progress waits for nothing unfinished. Warp i owns chunk kSW seg + i.
+// While a CTA works on one item, the tiles of its next item are already loading into the
+// other of two shared-memory buffers, and the ticket after that is being claimed.
+//   1. every warp recomputes its chunk's forward from the chunk's checkpoint: factors in
+//      registers, dr written in place of r, and the chunk's reverse map;
+//   2. warp 0 publishes the segment's map; the last warp forms the carry at the segment's
+//      end in a fixed order (bitwise reproducible): the carry published at the start of
+//      segment jc = seg + kFoldR + 1 (zero past the end), then the maps of segments
+//      jc-1 .. seg+1, so one link of a serial chain spans kFoldR + 1 segments;
+//   3. each warp applies the maps of the chunks after it to that carry and runs the reverse
+//      over its chunk: dk, dv in place of k, v, TMA-stored with dr; warp 0 publishes the
+//      carry at the segment's start where a segment further back starts from it; the
+//      chunks' partial sums of dw, du are added in a fixed order into per-segment partials.
+struct SegItem {
+  int seg, b, g;
+  int64_t bg;
+};
+
+__device__ __forceinline__ SegItem seg_item(unsigned tk, int64_t nbg, int nseg, int G) {
+  SegItem it;
+  const int back = int(tk / nbg);  // segments from the end
+  it.seg = nseg - 1 - back;
+  it.bg = int64_t(tk) - int64_t(back) * nbg;
+  it.b = int(it.bg / G);
+  it.g = int(it.bg - int64_t(it.b) * G);
+  return it;
+}
+
+template <bool GATE, bool DR>
+__global__ void __launch_bounds__(kSW * 32, 3)
+    wkv_bwd_seg_kernel(const __grid_constant__ TensorMaps4 in_maps,
+                       const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
+                       const float* __restrict__ w, const float* __restrict__ u, void* ws,
+                       unsigned* err) {
+  constexpr int kTile = kTT * 32;
+  constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
+  // Dynamic: [2 buffers][kSW warps][kNL tiles][kTile] floats.
+  extern __shared__ __align__(128) float dyn_tiles[];
+  __shared__ float4 sagg[kSW][32][2];           // the chunks' reverse maps
+  __shared__ float4 sfold[2 * kFoldR + 1][32];  // later segments' maps and carry
+  __shared__ float4 sxe[32];                    // the carry at the segment's end
+  __shared__ uint64_t bars[2][kSW];
+  __shared__ unsigned s_tk[2];
+  // The chunks' partial sums (-dw, du), in sfold's space (used at other times).
+  static_assert(2 * kFoldR + 1 >= kSW / 2, "spart must fit in sfold");
+  auto spart = reinterpret_cast<float2(*)[32]>(&sfold[0][0]);
+
+  const int G = (C + 31) >> 5;
+  const int64_t nbg = int64_t(B) * G;
+  const int nch = (T + kTT - 1) / kTT;
+  const int nseg = (nch + kSW - 1) / kSW;
+  const unsigned nitems = unsigned(nbg * nseg);
+  const BwdLayout lay = bwd_layout(ws, B, T, C);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto tile = [&](int buf, int i) { return dyn_tiles + ((buf * kSW + warp) * kNL + i) * kTile; };
+  // Lane 0 of each warp loads its own chunk of an item (no-op past the end of the sequence).
+  auto issue = [&](int buf, unsigned tk) {
+    const SegItem it = seg_item(tk, nbg, nseg, G);
+    const int ch = it.seg * kSW + warp;
+    if (ch < nch) {
+      uint64_t* bar = &bars[buf][warp];
+      mbar_arrive_expect_tx(bar, uint32_t(kNL) * kTile * sizeof(float));
+      for (int i = 0; i < kNL; ++i) tma_load_3d(tile(buf, i), &in_maps.m[i], bar, it.g << 5, ch * kTT, it.b);
+    }
+  };
+
+  if (lane == 0) {
+    mbar_init(&bars[0][warp], 1);
+    mbar_init(&bars[1][warp], 1);
+    mbar_fence_init();
+  }
+  if (threadIdx.x == 0) {
+    s_tk[0] = atomicAdd(lay.rticket, 1u);
+    s_tk[1] = atomicAdd(lay.rticket, 1u);
+  }
+  __syncthreads();
+  unsigned tk = s_tk[0], tk_next = s_tk[1];
+  __syncthreads();  // (s_tk is rewritten in the loop)
+  if (tk < nitems && lane == 0) issue(0, tk);
+  uint32_t phase = 0;  // bit buf: parity of this warp's next wait on buffer buf
+  int buf = 0;
+
+  while (tk < nitems) {
+    // The next item's tiles into the other buffer, once this warp's stores of the item
+    // before have read it; and the ticket after the next.
+    if (lane == 0) {
+      tma_store_wait_read<0>();
+      if (tk_next < nitems) issue(buf ^ 1, tk_next);
+    }
+    if (threadIdx.x == 0) s_tk[buf] = tk_next < nitems ? atomicAdd(lay.rticket, 1u) : nitems;
+
+    const SegItem it = seg_item(tk, nbg, nseg, G);
+    const int seg = it.seg, b = it.b, g = it.g;
+    const int c = (g << 5) + lane;
+    const bool valid = c < C;
+    const int ch = seg * kSW + warp;
+    const bool live = ch < nch;
+    const int t0 = ch * kTT;
+    const int64_t item0 = it.bg * nseg;
+    const int64_t item = item0 + seg;
+    float* K = tile(buf, 0) + lane;
+    float* V = tile(buf, 1) + lane;
+    float* R = tile(buf, 2) + lane;
+    const float* DY = tile(buf, kNL - 1) + lane;
+    const float4 ck = (live && valid) ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
+                                      : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
+    // The log2-scale of the state entering the next chunk (its checkpoint), see below.
+    const float2 nsc = (ch + 1 < nch && valid)
+                           ? *reinterpret_cast<const float2*>(
+                                 &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z)
+                           : make_float2(0.f, 0.f);
+    const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
+    const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+    const int rb = window_tokens(cp.w2, 128.f);
+
+    // ---- 1. forward recomputation and the chunk's reverse map ----
+    ChunkFactors f;
+    RevAgg A = rev_identity();
+    ChanState s;
+    s.a = ck.x;
+    s.b = ck.y;
+    s.Q = ck.z;
+    s.pl = ck.w;
+    if (live) {
+      mbar_wait(&bars[buf][warp], (phase >> buf) & 1u, err);
+      phase ^= 1u << buf;
+      __syncwarp();
+      A = fast ? chunk_forward_rb<GATE, DR, true>(s, cp, rb, K, V, R, DY, f)
+               : chunk_forward_rb<GATE, DR, false>(s, cp, rb, K, V, R, DY, f);
+    }
+    // The carry at this chunk's end comes scaled by the state entering the next chunk (its
+    // checkpoint); this chunk's own sums are scaled by its recomputed final state. Both are
+    // the same state reached by different orders of rounding: rescale by the exact ratio
+    // of the two scales (beta~ = beta 2^P) so the reverse sums stay consistent. The factor
+    // is folded into the chunk's map (E) for the chunks before it.
+    const float rme = (ch + 1 < nch) ? ex2(fminf((s.Q - nsc.x) + (s.pl - nsc.y), 64.f)) : 1.f;
+    A.E *= rme;
+    put_agg(&sagg[warp][lane][0], A);
+    __syncthreads();
+
+    // ---- 2. the segment's map; the carry at its end ----
+    if (warp == 0 && seg > 0) {  // the segment's map, for the segments before it
+      RevAgg M = get_agg(sagg[kSW - 1][lane][0], sagg[kSW - 1][lane][1]);
+#pragma unroll
+      for (int i = kSW - 2; i >= 0; --i) M = rev_compose(get_agg(sagg[i][lane][0], sagg[i][lane][1]), M);
+      put_agg(&lay.rmap[(item * 32 + lane) * 2], M);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(&lay.rflags[item], 1u);
+    }
+    if (warp == kSW - 1) {
+      const int jc = min(nseg, seg + kFoldR + 1);
+      const int m = jc - 1 - seg;  // maps to apply
+      unsigned fl = 1;
+      if (lane < m) fl = wait_flag(&lay.rflags[item0 + seg + 1 + lane], 1u, kWaitLimitNs, err);
+      if (lane == 31 && jc < nseg) fl = wait_flag(&lay.rflags[item0 + jc], 2u, kWaitLimitNs, err);
+      const bool ok = __all_sync(0xffffffffu, fl != 0);
+      RevCarry X{0.f, 0.f, 0.f, 0.f};
+      if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
+        // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
+        for (int l = 0; l < 2 * m; ++l)  // map of segment seg + 1 + l / 2, half l % 2
+          sfold[l][lane] = __ldcg(&lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
+        if (jc < nseg) {
+          const float4 q = __ldcg(&lay.carry[(item0 + jc) * 32 + lane]);
+          X = RevCarry{q.x, q.y, q.z, q.w};
+        }
+        __syncwarp();
+        for (int l = m - 1; l >= 0; --l)
+          X = rev_apply(get_agg(sfold[2 * l][lane], sfold[2 * l + 1][lane]), X);
+      }
+      sxe[lane] = make_float4(X.b, X.g, X.bd, X.gd);
+    }
+    __syncthreads();
+
+    // ---- 3. carries, reverse over the chunks ----
+    const float4 xe = sxe[lane];
+    RevCarry X{xe.x, xe.y, xe.z, xe.w};
+    for (int i = kSW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
+    if (warp == 0 && seg > kFoldR) {  // segment seg - kFoldR - 1 starts from this carry
+      const RevCarry X0 = rev_apply(A, X);
+      lay.carry[item * 32 + lane] = make_float4(X0.b, X0.g, X0.bd, X0.gd);
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) st_release(&lay.rflags[item], 2u);
+    }
+    float2 part = make_float2(0.f, 0.f);
+    if (live) {
+      part = chunk_reverse(f, RevCarry{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme}, K, V);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        for (int i = 0; i < (DR ? 3 : 2); ++i) tma_store_3d(&out_maps.m[i], tile(buf, i), g << 5, t0, b);
+        tma_store_commit();
+      }
+    }
+    spart[warp][lane] = part;
+    __syncthreads();
+    if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
+      float sw = 0.f, su = 0.f;
+#pragma unroll
+      for (int i = 0; i < kSW; ++i) {
+        sw += spart[i][lane].x;
+        su += spart[i][lane].y;
+      }
+      lay.pdw[(int64_t(b) * nseg + seg) * C + c] = sw;
+      lay.pdu[(int64_t(b) * nseg + seg) * C + c] = su;
+    }
+    tk = tk_next;
+    tk_next = s_tk[buf];
+    buf ^= 1;
+  }
+  if (lane == 0) tma_store_wait_all();
+}
+
+// ---- 3. reduction over batch rows and segments, fixed order -------------------------------
+// Block (32, kRS): lane x owns a channel; slice y sums the rows y, y + kRS, ... in order,
+// then slice 0 adds the slices' sums in order. Same order on every call: deterministic.
+constexpr int kRS = 32;
+__global__ void __launch_bounds__(32 * kRS) wkv_bwd_reduce_kernel(int B, int C, const void* ws,
+                                                                 int T, float* dw, float* du) {
+  __shared__ float2 sp[kRS][33];
+  const int c = blockIdx.x * 32 + threadIdx.x;
   const BwdLayout lay = bwd_layout(const_cast<void*>(ws), B, T, C);
+  const int64_t rows = int64_t(B) * bwd_nseg(T);
   float sw = 0.f, su = 0.f;
-  for (int b = 0; b < B; ++b) {
-    sw += lay.pdw[int64_t(b) * C + c];
-    su += lay.pdu[int64_t(b) * C + c];
+  if (c < C) {
+#pragma unroll 8
+    for (int64_t i = threadIdx.y; i < rows; i += kRS) {
+      sw += lay.pdw[i * C + c];
+      su += lay.pdu[i * C + c];
+    }
   }
-  dw[c] = sw;
-  du[c] = su;
+  sp[threadIdx.y][threadIdx.x] = make_float2(sw, su);
+  __syncthreads();
+  if (threadIdx.y == 0 && c < C) {
+    float tw = 0.f, tu = 0.f;
+    for (int y = 0; y < kRS; ++y) {
+      tw += sp[y][threadIdx.x].x;
+      tu += sp[y][threadIdx.x].y;
+    }
+    dw[c] = tw;
+    du[c] = tu;
+  }
 }
 
-size_t bwd_main_smem() { return (8 + 6) * kTT * 32 * sizeof(float) + 2 * sizeof(uint64_t); }
+size_t bwd_main_smem() {
+  return (4 * kMS + 6) * kTT * 32 * sizeof(float) + kMS * sizeof(uint64_t);
+}
 
 template <bool TMA, bool GATE, bool DR>
 int launch_main(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
@@ -383,6 +1005,26 @@ int launch_main(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
   const int64_t grid = a.B * ((a.C + 31) / 32);
   kern<<<unsigned(grid), 32, smem, stream>>>(in, out, a.k, a.v, a.r, a.dy, a.dk, a.dv, a.dr,
                                              int(a.B), int(a.T), int(a.C), a.w, a.u, a.ws, a.err);
+  return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+template <bool GATE, bool DR>
+int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, int64_t nitems,
+               cudaStream_t stream) {
+  auto kern = wkv_bwd_seg_kernel<GATE, DR>;
+  const size_t smem = 2 * size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return WKV_ERR_CUDA;
+  // Persistent: as many CTAs as fit at once (never more than there are items).
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSW * 32, smem) != cudaSuccess)
+    return WKV_ERR_CUDA;
+  const int64_t grid = std::min<int64_t>(nitems, int64_t(std::max(1, per_sm)) * sms);
+  kern<<<unsigned(grid), kSW * 32, smem, stream>>>(in, out, int(a.B), int(a.T), int(a.C), a.w,
+                                                    a.u, a.ws, a.err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -401,18 +1043,34 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     ck.m[0] = in.m[0];
     ck.m[1] = in.m[1];
   }
-  wkv_bwd_ckpt_kernel<TMA><<<unsigned(grid), 32, 0, stream>>>(ck, a.k, a.v, int(a.B), int(a.T),
-                                                              int(a.C), a.w, a.ws, a.err);
-  if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
   int rc;
-  if (a.r)
-    rc = a.dr ? launch_main<TMA, true, true>(a, in, out, stream)
-              : launch_main<TMA, true, false>(a, in, out, stream);
-  else
-    rc = launch_main<TMA, false, false>(a, in, out, stream);
+  if (TMA) {
+    // Time-parallel checkpoints and reverse: the chain flags and the tickets start at zero.
+    const int64_t nitems = grid * bwd_nseg(a.T);
+    if (nitems >= (int64_t(1) << 31)) return WKV_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(a.ws, 0, bwd_flag_bytes(a.B, a.T, a.C), stream) != cudaSuccess)
+      return WKV_ERR_CUDA;
+    wkv_bwd_ckpt_seg_kernel<<<unsigned(nitems), kSW * 32, 0, stream>>>(
+        ck, int(a.B), int(a.T), int(a.C), a.w, a.ws, a.err);
+    if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
+    if (a.r)
+      rc = a.dr ? launch_seg<true, true>(a, in, out, nitems, stream)
+                : launch_seg<true, false>(a, in, out, nitems, stream);
+    else
+      rc = launch_seg<false, false>(a, in, out, nitems, stream);
+  } else {
+    wkv_bwd_ckpt_kernel<TMA><<<unsigned(grid), 32, 0, stream>>>(ck, a.k, a.v, int(a.B), int(a.T),
+                                                                int(a.C), a.w, a.ws, a.err);
+    if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
+    if (a.r)
+      rc = a.dr ? launch_main<TMA, true, true>(a, in, out, stream)
+                : launch_main<TMA, true, false>(a, in, out, stream);
+    else
+      rc = launch_main<TMA, false, false>(a, in, out, stream);
+  }
   if (rc) return rc;
-  wkv_bwd_reduce_kernel<<<unsigned((a.C + 127) / 128), 128, 0, stream>>>(int(a.B), int(a.C), a.ws,
-                                                                        int(a.T), a.dw, a.du);
+  wkv_bwd_reduce_kernel<<<unsigned((a.C + 31) / 32), dim3(32, kRS), 0, stream>>>(
+      int(a.B), int(a.C), a.ws, int(a.T), a.dw, a.du);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 

@@ -85,6 +85,33 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Flag words of the look-back scans: release on publish, acquire on observe (gpu scope).
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Spin until *flag >= want (lane 0 of a warp only); gives up after wait_ns, flagging err.
+// Returns the flag value seen (0 when it gave up).
+__device__ __forceinline__ unsigned wait_flag(const unsigned* flag, unsigned want,
+                                              uint64_t wait_ns, unsigned* err) {
+  unsigned f = ld_acquire(flag);
+  if (f >= want) return f;
+  const uint64_t start = global_ns();
+  while ((f = ld_acquire(flag)) < want) {
+    if (global_ns() - start > wait_ns) {
+      atomicOr(err, kErrTimeout);
+      return 0;
+    }
+    __nanosleep(64);
+  }
+  return f;
+}
+
 // Wait limit for every spin in this library: about two seconds of wall time.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

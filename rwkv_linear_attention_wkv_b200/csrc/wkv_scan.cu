@@ -51,52 +51,6 @@ constexpr int kLS = WKV_SCAN_LS;   // tokens per sub-chunk
 constexpr int kSeg = kW * kLS;
 constexpr int64_t kChunkBelowChannels = WKV_SCAN_MIN_CH;
 
-struct Agg {  // scaled numerator, denominator, log2-scale as an exact pair
-  float a, b, ph, pl;
-};
-
-__device__ __forceinline__ Agg agg_empty() { return Agg{0.f, 0.f, kEmptyLogScale, 0.f}; }
-
-// X (+) Y where Y spans `len` tokens after X.
-__device__ __forceinline__ Agg combine(const Agg& X, const Agg& Y, float len, float w2) {
-  float xh, xl;
-  decay_pair(X.ph, X.pl, len, w2, xh, xl);
-  const float d = (xh - Y.ph) + (xl - Y.pl);
-  const float f = ex2(-fabsf(d));
-  Agg r;
-  if (d > 0.f) {
-    r.a = fmaf(f, Y.a, X.a);
-    r.b = fmaf(f, Y.b, X.b);
-    r.ph = xh;
-    r.pl = xl;
-  } else {
-    r.a = fmaf(f, X.a, Y.a);
-    r.b = fmaf(f, X.b, Y.b);
-    r.ph = Y.ph;
-    r.pl = Y.pl;
-  }
-  return r;
-}
-
-__device__ __forceinline__ Agg to_agg(const ChanState& s) { return Agg{s.a, s.b, s.Q, s.pl}; }
-__device__ __forceinline__ ChanState to_state(const Agg& g) {
-  ChanState s;
-  s.a = g.a;
-  s.b = g.b;
-  s.Q = g.ph;
-  s.pl = g.pl;
-  return s;
-}
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 struct ScanLayout {
   unsigned* ticket;
   unsigned* flags;  // [nbg * nseg]: 0 none, 1 aggregate, 2 inclusive prefix

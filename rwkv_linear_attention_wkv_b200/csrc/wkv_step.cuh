@@ -178,4 +178,49 @@ __device__ __forceinline__ int window_tokens(float w2, float limit) {
   return (16.f * m <= limit) ? 16 : ((4.f * m <= limit) ? 4 : 1);
 }
 
+// ---- span aggregates ------------------------------------------------------------------
+// Because the decay e^{-w} does not depend on time, the state after two adjacent spans is an
+// associative combination of the first span's state and the second span's own aggregate
+// (its state from the empty state):
+//   X (+) Y over a span Y of L tokens:  scale_X' = scale_X - L w2 (log2),
+//   (a, b) = (a_X 2^{scale_X' - s} + a_Y 2^{scale_Y - s}, same for b),  s = max(scale_X', scale_Y)
+// (one exponential: one of the two factors is 1). Scales are exact float pairs (hi, lo) so
+// that a long chain of combinations does not drift.
+struct Agg {  // scaled numerator, denominator, log2-scale as an exact pair
+  float a, b, ph, pl;
+};
+
+__device__ __forceinline__ Agg agg_empty() { return Agg{0.f, 0.f, kEmptyLogScale, 0.f}; }
+
+// X (+) Y where Y spans `len` tokens after X.
+__device__ __forceinline__ Agg combine(const Agg& X, const Agg& Y, float len, float w2) {
+  float xh, xl;
+  decay_pair(X.ph, X.pl, len, w2, xh, xl);
+  const float d = (xh - Y.ph) + (xl - Y.pl);
+  const float f = ex2(-fabsf(d));
+  Agg r;
+  if (d > 0.f) {
+    r.a = fmaf(f, Y.a, X.a);
+    r.b = fmaf(f, Y.b, X.b);
+    r.ph = xh;
+    r.pl = xl;
+  } else {
+    r.a = fmaf(f, X.a, Y.a);
+    r.b = fmaf(f, X.b, Y.b);
+    r.ph = Y.ph;
+    r.pl = Y.pl;
+  }
+  return r;
+}
+
+__device__ __forceinline__ Agg to_agg(const ChanState& s) { return Agg{s.a, s.b, s.Q, s.pl}; }
+__device__ __forceinline__ ChanState to_state(const Agg& g) {
+  ChanState s;
+  s.a = g.a;
+  s.b = g.b;
+  s.Q = g.ph;
+  s.pl = g.pl;
+  return s;
+}
+
 }  // namespace wkv

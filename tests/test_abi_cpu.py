@@ -80,10 +80,16 @@ def test_decode_and_backward_argument_checks(W):
 
 
 def test_backward_workspace_size(W):
-    # checkpoints (a, b, Q, pl) per 32-token chunk and channel, plus dw, du partials [B, C]
+    # Chain flags (16 bytes of tickets, then two words per segment item), the forward state
+    # (a, b, Q, pl) entering every 16-token chunk, per-segment partials of dw and du, and per
+    # segment item of 4 chunks and lane: its forward aggregate (1 float4), reverse map
+    # (2 float4) and reverse carry (1 float4).
     def a256(x):
         return (x + 255) // 256 * 256
     for B, T, C in ((16, 1024, 768), (1, 33, 5), (3, 1, 4096)):
-        nch = (T + 31) // 32
-        want = a256(B * nch * C * 16) + 2 * a256(B * C * 4)
+        nch = (T + 15) // 16
+        nseg = (nch + 3) // 4
+        nitems = B * ((C + 31) // 32) * nseg
+        want = (a256(16 + 8 * nitems) + a256(B * nch * C * 16) + 2 * a256(B * nseg * C * 4)
+                + a256(nitems * 32 * 16) + a256(nitems * 32 * 32) + a256(nitems * 32 * 16))
         assert W.wkv_backward_workspace_bytes(B, T, C) == want
