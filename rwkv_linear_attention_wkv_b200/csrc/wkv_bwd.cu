@@ -52,7 +52,7 @@ constexpr int kSW = 4;    // chunks (warps) per segment of the time-parallel pas
 // Segments whose results a segment folds in directly before taking a carry from further
 // away (which makes one link of a serial chain per kFoldF / kFoldR + 1 segments): in the
 // checkpoint pass (forward) and the reverse pass.
-constexpr int kFoldF = 16;
+constexpr int kFoldF = 8;
 constexpr int kFoldR = 5;
 
 struct BwdLayout {
@@ -61,10 +61,11 @@ struct BwdLayout {
   float* pdu;        // [B, nseg, C] per-segment partial sums of du
   unsigned* fticket;  // segment tickets of the checkpoint pass (forward chain)
   unsigned* rticket;  // segment tickets of the reverse pass (reverse chain)
-  unsigned* fflags;   // [nbg * nseg]: 1 once the segment's aggregate is published, 2 once the
-                      // state entering it (its first checkpoint) is written
+  unsigned* fflags;   // [nbg * nseg']: 1 once the checkpoint segment's aggregate is published,
+                      // 2 once the state entering it (its first checkpoint) is written
+                      // (nseg' <= nseg checkpoint segments of kSW kCK chunks)
   unsigned* rflags;   // [nbg * nseg]: 1 once the segment's reverse map is published, 2 its carry
-  float4* fagg;      // [nbg * nseg, 32]: the segment's forward aggregate (a, b, ph, pl)
+  float4* fagg;      // [nbg * nseg', 32]: the checkpoint segment's aggregate (a, b, ph, pl)
   float4* rmap;      // [nbg * nseg, 32, 2]: the segment's reverse map (see RevAgg)
   float4* carry;     // [nbg * nseg, 32]: (beta, gamma, betad, gammad) at the segment start
 };
@@ -284,22 +285,50 @@ __device__ __forceinline__ void absorb_indep(ChanState& s, const ChanParams& cp,
   s.b = fmaf(e1, s.b, e2);
 }
 
-// Time-parallel form (TMA shapes). One CTA per (segment of kSW chunks, batch row, 32-channel
-// group), warp i on chunk kSW seg + i; CTAs take segments in ticket order from the first on,
-// so every segment a CTA waits for belongs to a CTA that started earlier. Each warp folds its
-// chunk's k, v into the chunk's aggregate from the empty state. Before its own chunk, the
-// last warp forms the state entering the segment, in a fixed order (bitwise reproducible):
-// the state entering segment j0 = max(0, seg - kFoldF) (its first checkpoint), then the
-// published aggregates of segments j0 .. seg-1; so one link of a serial chain spans kFoldF
-// segments. After one barrier each warp combines that state with the aggregates of the
-// chunks before its own and writes its chunk's checkpoint; warp 0 publishes the segment's
-// aggregate. One pass, 8 bytes of HBM reads per element.
-__global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
+// Time-parallel form (TMA shapes). One CTA per (checkpoint segment of kSW x kCK chunks,
+// batch row, 32-channel group), warp i on chunks kCK i .. kCK i + kCK - 1 of the segment;
+// CTAs take segments in ticket order from the first on, so every segment a CTA waits for
+// belongs to a CTA that started earlier. Each warp folds its chunks' k, v into each chunk's
+// aggregate from the empty state. Warp 0 publishes the segment's aggregate; the last warp
+// forms the state entering the segment in a fixed order (bitwise reproducible): the state
+// entering segment j0 = max(0, seg - kFoldF) (its first checkpoint), then the published
+// aggregates of segments j0 .. seg-1, so one link of a serial chain spans kFoldF segments.
+// After a barrier each warp combines that state with the aggregates of the chunks before
+// its own and writes its chunks' checkpoints. One pass, 8 bytes of HBM reads per element.
+constexpr int kCK = 2;  // chunks per warp in the checkpoint pass
+
+// Aggregate of one chunk of n tokens from the empty state (windows of RB tokens).
+template <int RB>
+__device__ __forceinline__ Agg chunk_aggregate(const float* K, const float* V, int n,
+                                               const ChanParams& cp) {
+  ChanState s = empty_state();
+  if (n == kTT) {
+#pragma unroll
+    for (int t = 0; t < kTT; ++t) {
+      absorb_indep(s, cp, float(t % RB + 1), K[t * 32], V[t * 32]);
+      if ((t + 1) % RB == 0) wkv_rebase(s, float(RB) * cp.w2);
+    }
+  } else {
+    int j = 0;
+    for (int t = 0; t < n; ++t) {
+      absorb_indep(s, cp, float(j + 1), K[t * 32], V[t * 32]);
+      if (++j == RB) {
+        wkv_rebase(s, float(RB) * cp.w2);
+        j = 0;
+      }
+    }
+    if (j) wkv_rebase_partial(s, j, cp.w2);
+  }
+  return to_agg(s);
+}
+
+__global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
     const __grid_constant__ TensorMaps4 maps, int B, int T, int C, const float* __restrict__ w,
     void* ws, unsigned* err) {
   constexpr int kTile = kTT * 32;
-  __shared__ __align__(128) float tiles[kSW][2][kTile];  // k, v per warp
-  __shared__ float4 sagg[kSW][32];
+  constexpr int kSegC = kSW * kCK;  // chunks per checkpoint segment
+  __shared__ __align__(128) float tiles[kSW][kCK][2][kTile];  // k, v of each warp's chunks
+  __shared__ float4 sagg[kSegC][32];
   __shared__ float4 sfold[kFoldF][32];  // earlier segments' aggregates
   __shared__ float4 sin_[32];           // the state entering the segment
   __shared__ uint64_t bars[kSW];
@@ -308,7 +337,7 @@ __global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
   const int G = (C + 31) >> 5;
   const int64_t nbg = int64_t(B) * G;
   const int nch = (T + kTT - 1) / kTT;
-  const int nseg = (nch + kSW - 1) / kSW;
+  const int nseg = (nch + kSegC - 1) / kSegC;
   const BwdLayout lay = bwd_layout(ws, B, T, C);
   if (threadIdx.x == 0) s_ticket = atomicAdd(lay.fticket, 1u);
   __syncthreads();
@@ -320,8 +349,7 @@ __global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = (g << 5) + lane;
   const bool valid = c < C;
-  const int ch = seg * kSW + warp;
-  const int n = max(0, min(kTT, T - ch * kTT));  // tokens of this warp's chunk
+  const int ch0 = seg * kSegC + warp * kCK;  // this warp's first chunk
   const int64_t item0 = bg * nseg;
   const int64_t item = item0 + seg;
   float4* ck = lay.ckpt + int64_t(b) * nch * C + c;  // checkpoint of chunk i at ck[i * C]
@@ -330,34 +358,44 @@ __global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
   if (lane == 0) {
     mbar_init(bar, 1);
     mbar_fence_init();
-    if (n > 0) {
-      mbar_arrive_expect_tx(bar, 2u * kTile * sizeof(float));
-      tma_load_3d(&tiles[warp][0][0], &maps.m[0], bar, g << 5, ch * kTT, b);
-      tma_load_3d(&tiles[warp][1][0], &maps.m[1], bar, g << 5, ch * kTT, b);
+    const int nc = max(0, min(kCK, nch - ch0));  // chunks of this warp
+    if (nc > 0) {
+      mbar_arrive_expect_tx(bar, uint32_t(nc) * 2u * kTile * sizeof(float));
+      for (int q = 0; q < nc; ++q) {
+        tma_load_3d(&tiles[warp][q][0][0], &maps.m[0], bar, g << 5, (ch0 + q) * kTT, b);
+        tma_load_3d(&tiles[warp][q][1][0], &maps.m[1], bar, g << 5, (ch0 + q) * kTT, b);
+      }
     }
   }
   __syncwarp();
   const ChanParams cp = chan_params(valid ? w[c] : 1.f, 0.f);
   const int rb = window_tokens(cp.w2, 128.f);
 
-  // ---- the chunk's aggregate from the empty state ----
-  Agg A = agg_empty();
-  if (n > 0) {
-    mbar_wait(bar, 0, err);
-    __syncwarp();
-    ChanState s = empty_state();
-    int j = 0;
-    for (int t = 0; t < n; ++t) {
-      absorb_indep(s, cp, float(j + 1), tiles[warp][0][t * 32 + lane], tiles[warp][1][t * 32 + lane]);
-      if (++j == rb) {
-        wkv_rebase(s, float(rb) * cp.w2);
-        j = 0;
-      }
-    }
-    if (j) wkv_rebase_partial(s, j, cp.w2);
-    A = to_agg(s);
+  // The fold's inputs (below) are usually published long before they are needed: read
+  // their flags now (relaxed, not waited for) and only wait later if one was not.
+  const int j0 = max(0, seg - kFoldF);
+  const int mfold = seg - j0;  // aggregates to fold
+  unsigned fearly = 0;
+  if (warp == kSW - 1) {
+    if (lane < mfold) fearly = ld_relaxed(&lay.fflags[item0 + j0 + lane]);
+    if (lane == 31 && j0 > 0) fearly = ld_relaxed(&lay.fflags[item0 + j0]);
   }
-  sagg[warp][lane] = make_float4(A.a, A.b, A.ph, A.pl);
+
+  // ---- the chunks' aggregates from the empty state ----
+  if (ch0 < nch) mbar_wait(bar, 0, err);
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < kCK; ++q) {
+    const int n = max(0, min(kTT, T - (ch0 + q) * kTT));  // tokens of the chunk
+    Agg A = agg_empty();
+    if (n > 0) {
+      const float* K = &tiles[warp][q][0][lane];
+      const float* V = &tiles[warp][q][1][lane];
+      A = rb == 16 ? chunk_aggregate<16>(K, V, n, cp)
+                   : (rb == 4 ? chunk_aggregate<4>(K, V, n, cp) : chunk_aggregate<1>(K, V, n, cp));
+    }
+    sagg[warp * kCK + q][lane] = make_float4(A.a, A.b, A.ph, A.pl);
+  }
   __syncthreads();
 
   // ---- the segment's aggregate, for the segments after it ----
@@ -365,57 +403,67 @@ __global__ void __launch_bounds__(kSW * 32, 8) wkv_bwd_ckpt_seg_kernel(
   if (warp == 0 && seg + 1 < nseg) {
     Agg S = agg_empty();
 #pragma unroll
-    for (int i = 0; i < kSW; ++i) {
+    for (int i = 0; i < kSegC; ++i) {
       const float4 q = sagg[i][lane];
       S = combine(S, Agg{q.x, q.y, q.z, q.w}, float(kTT), cp.w2);  // all chunks full
     }
     lay.fagg[item * 32 + lane] = make_float4(S.a, S.b, S.ph, S.pl);
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release(&lay.fflags[item], 1u);
+    warp_publish(&lay.fflags[item], 1u);
   }
   // ---- the state entering the segment (last warp; the aggregate above does not wait) ----
   if (warp == kSW - 1) {
-    const int j0 = max(0, seg - kFoldF);
-    const int m = seg - j0;  // aggregates to fold
-    unsigned fl = 1;
-    if (lane < m) fl = wait_flag(&lay.fflags[item0 + j0 + lane], 1u, kWaitLimitNs, err);
-    if (lane == 31 && j0 > 0) fl = wait_flag(&lay.fflags[item0 + j0], 2u, kWaitLimitNs, err);
-    const bool ok = __all_sync(0xffffffffu, fl != 0);
+    const int m = mfold;
+    const unsigned want = lane < m ? 1u : ((lane == 31 && j0 > 0) ? 2u : 0u);
+    // Each lane completes the acquire of its own flag before the warp barrier; the barrier
+    // then orders every lane's fetch below after all of them.
+    fence_acquire();
+    bool ok = true;
+    if (!__all_sync(0xffffffffu, fearly >= want)) {
+      unsigned fl = 1;
+      if (want != 0 && fearly < want)
+        fl = wait_flag(lane < m ? &lay.fflags[item0 + j0 + lane] : &lay.fflags[item0 + j0], want,
+                       kWaitLimitNs, err);
+      ok = __all_sync(0xffffffffu, fl != 0);
+    }
     Agg X = agg_empty();
     if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
       // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
       for (int l = 0; l < m; ++l) sfold[l][lane] = __ldcg(&lay.fagg[(item0 + j0 + l) * 32 + lane]);
       if (j0 > 0 && valid) {
-        const float4 q = __ldcg(&ck[int64_t(j0) * kSW * C]);
+        const float4 q = __ldcg(&ck[int64_t(j0) * kSegC * C]);
         X = Agg{q.x, q.y, q.z, q.w};
       }
       __syncwarp();
       for (int l = 0; l < m; ++l) {
         const float4 a = sfold[l][lane];
-        X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kSW * kTT), cp.w2);
+        X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kSegC * kTT), cp.w2);
       }
     }
     sin_[lane] = make_float4(X.a, X.b, X.ph, X.pl);
   }
-
   __syncthreads();
 
   // ---- checkpoints ----
   {
     const float4 q = sin_[lane];
     Agg X{q.x, q.y, q.z, q.w};
-    for (int i = 0; i < warp; ++i) {  // chunks before this one (full)
+    for (int i = 0; i < warp * kCK; ++i) {  // chunks before this warp's (full)
       const float4 a = sagg[i][lane];
       X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kTT), cp.w2);
     }
-    if (n > 0 && valid) ck[int64_t(ch) * C] = make_float4(X.a, X.b, X.ph, X.pl);
+#pragma unroll
+    for (int q2 = 0; q2 < kCK; ++q2) {
+      const int chq = ch0 + q2;
+      if (chq < nch) {
+        if (valid) ck[int64_t(chq) * C] = make_float4(X.a, X.b, X.ph, X.pl);
+        if (q2 + 1 < kCK) {
+          const float4 a = sagg[warp * kCK + q2][lane];
+          X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kTT), cp.w2);
+        }
+      }
+    }
   }
-  if (warp == 0 && first) {  // the first checkpoint is written: release it
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release(&lay.fflags[item], 2u);
-  }
+  if (warp == 0 && first) warp_publish(&lay.fflags[item], 2u);  // the first checkpoint is written
 }
 
 // ---- 2. reverse pass ---------------------------------------------------------------------
@@ -632,22 +680,23 @@ __device__ __forceinline__ RevAgg get_agg(float4 x, float4 y) {
   return RevAgg{x.x, y.y, x.y, x.z, x.w, y.x};
 }
 
-// Per-token factors of one chunk from the forward recomputation, kept in registers (every
-// index is a compile-time constant after unrolling). e1/e2: one of them is 1, the other is
-// fe[t]; bit t of `tok` says which (set: the token's own term dominated, e1 = fe[t],
-// e2 = 1). inj and cur already carry the token's dy.
+// Per-token factors of one chunk from the forward recomputation. e1/e2: one of them is 1,
+// the other is fe[t]; bit t of `tok` says which (set: the token's own term dominated,
+// e1 = fe[t], e2 = 1). inj carries the token's dy. fe and inj stay in registers (every
+// index is a compile-time constant after unrolling); wkv and cur (h e^{u+k}, with dy) go to
+// shared memory in place of k and dy, which the reverse no longer needs.
 struct ChunkFactors {
-  float fe[kTT], inj[kTT], cur[kTT], wkv[kTT];
+  float fe[kTT], inj[kTT];
   unsigned tok;
 };
 
 // Forward recomputation of one chunk of kTT tokens from its entering state s (left holding
-// the state after the chunk): fills the per-token factors, writes dr in place of r (DR),
-// and returns the chunk's reverse map (its sums from a zero carry, composed token by token
-// in time order).
+// the state after the chunk): fills the per-token factors (wkv into K, cur into DY), writes
+// dr in place of r (DR), and returns the chunk's reverse map (its sums from a zero carry,
+// composed token by token in time order).
 template <bool GATE, bool DR, bool FASTOUT, int RB>
-__device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& cp, const float* K,
-                                                const float* V, float* R, const float* DY,
+__device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& cp, float* K,
+                                                const float* V, float* R, float* DY,
                                                 ChunkFactors& f) {
   static_assert(kTT % RB == 0, "windows must tile the chunk");
   RevAgg A = rev_identity();
@@ -690,8 +739,8 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
     f.fe[t] = e;
     f.tok |= cnd ? (1u << t) : 0u;
     f.inj[t] = inj;
-    f.cur[t] = h * kc;
-    f.wkv[t] = wk;
+    K[t * 32] = wk;
+    DY[t * 32] = h * kc;
     if (DR) R[t * 32] = gy * wk * sig * (1.f - sig);  // dr in place of r
     // Compose the single-token map (E = e1, L = 1, l_beta = inj, l_gamma = inj wkv) after A.
     const float ej = A.E * inj;
@@ -710,25 +759,25 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
 
 template <bool GATE, bool DR, bool FASTOUT>
 __device__ __forceinline__ RevAgg chunk_forward_rb(ChanState& s, const ChanParams& cp, int rb,
-                                                   const float* K, const float* V, float* R,
-                                                   const float* DY, ChunkFactors& f) {
+                                                   float* K, const float* V, float* R, float* DY,
+                                                   ChunkFactors& f) {
   if (rb == 16) return chunk_forward<GATE, DR, FASTOUT, 16>(s, cp, K, V, R, DY, f);
   if (rb == 4) return chunk_forward<GATE, DR, FASTOUT, 4>(s, cp, K, V, R, DY, f);
   return chunk_forward<GATE, DR, FASTOUT, 1>(s, cp, K, V, R, DY, f);
 }
 
-// Reverse over one chunk from the carry X at its end: dk, dv replace k, v in shared memory;
-// returns the chunk's partial sums of -dw (.x) and du (.y).
+// Reverse over one chunk from the carry X at its end: dk, dv replace wkv (in K), v in shared
+// memory; returns the chunk's partial sums of -dw (.x) and du (.y).
 __device__ __forceinline__ float2 chunk_reverse(const ChunkFactors& f, RevCarry X, float* K,
-                                                float* V) {
+                                                float* V, const float* CUR) {
   float dw_acc = 0.f, du_acc = 0.f;
 #pragma unroll
   for (int t = kTT - 1; t >= 0; --t) {
-    const float vv = V[t * 32];
+    const float vv = V[t * 32], wk = K[t * 32], cur = CUR[t * 32];
     const bool dom = (f.tok >> t) & 1u;
     const float e1 = dom ? f.fe[t] : 1.f;
     const float e2 = dom ? 1.f : f.fe[t];
-    const float wk = f.wkv[t], inj = f.inj[t], cur = f.cur[t];
+    const float inj = f.inj[t];
     const float vm = vv - wk;
     V[t * 32] = fmaf(e2, X.b, cur);                            // dv
     K[t * 32] = fmaf(cur, vm, e2 * fmaf(vv, X.b, -X.g));       // dk
@@ -742,52 +791,34 @@ __device__ __forceinline__ float2 chunk_reverse(const ChunkFactors& f, RevCarry 
   return make_float2(-dw_acc, du_acc);
 }
 
-// Persistent CTAs of kSW warps; each takes segment items (a segment of kSW chunks of one
-// batch row and 32-channel group) in ticket order from the LAST segment backward, so every
-// segment an item waits for has a smaller ticket: it is done or in progress, and the
-// smallest item in progress waits for nothing unfinished. Warp i owns chunk kSW seg + i.
-// While a CTA works on one item, the tiles of its next item are already loading into the
-// other of two shared-memory buffers, and the ticket after that is being claimed.
-//   1. every warp recomputes its chunk's forward from the chunk's checkpoint: factors in
-//      registers, dr written in place of r, and the chunk's reverse map;
+// One CTA per (segment of kSW chunks, batch row, 32-channel group); warp i owns chunk
+// kSW seg + i. CTAs take segments in ticket order from the LAST segment backward, so every
+// segment a CTA waits for belongs to a CTA that started earlier: the waits always end.
+//   1. every warp TMA-loads its chunk's k, v, (r,) dy tiles and recomputes the forward from
+//      the chunk's checkpoint: factors, dr in place of r, and the chunk's reverse map;
 //   2. warp 0 publishes the segment's map; the last warp forms the carry at the segment's
 //      end in a fixed order (bitwise reproducible): the carry published at the start of
 //      segment jc = seg + kFoldR + 1 (zero past the end), then the maps of segments
 //      jc-1 .. seg+1, so one link of a serial chain spans kFoldR + 1 segments;
 //   3. each warp applies the maps of the chunks after it to that carry and runs the reverse
-//      over its chunk: dk, dv in place of k, v, TMA-stored with dr; warp 0 publishes the
+//      over its chunk: dk, dv in place of wkv, v, TMA-stored with dr; warp 0 publishes the
 //      carry at the segment's start where a segment further back starts from it; the
 //      chunks' partial sums of dw, du are added in a fixed order into per-segment partials.
-struct SegItem {
-  int seg, b, g;
-  int64_t bg;
-};
-
-__device__ __forceinline__ SegItem seg_item(unsigned tk, int64_t nbg, int nseg, int G) {
-  SegItem it;
-  const int back = int(tk / nbg);  // segments from the end
-  it.seg = nseg - 1 - back;
-  it.bg = int64_t(tk) - int64_t(back) * nbg;
-  it.b = int(it.bg / G);
-  it.g = int(it.bg - int64_t(it.b) * G);
-  return it;
-}
-
 template <bool GATE, bool DR>
-__global__ void __launch_bounds__(kSW * 32, 3)
+__global__ void __launch_bounds__(kSW * 32, 5)
     wkv_bwd_seg_kernel(const __grid_constant__ TensorMaps4 in_maps,
                        const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
                        const float* __restrict__ w, const float* __restrict__ u, void* ws,
                        unsigned* err) {
   constexpr int kTile = kTT * 32;
   constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
-  // Dynamic: [2 buffers][kSW warps][kNL tiles][kTile] floats.
+  // Dynamic: [kSW warps][kNL tiles][kTile] floats.
   extern __shared__ __align__(128) float dyn_tiles[];
   __shared__ float4 sagg[kSW][32][2];           // the chunks' reverse maps
   __shared__ float4 sfold[2 * kFoldR + 1][32];  // later segments' maps and carry
   __shared__ float4 sxe[32];                    // the carry at the segment's end
-  __shared__ uint64_t bars[2][kSW];
-  __shared__ unsigned s_tk[2];
+  __shared__ uint64_t bars[kSW];
+  __shared__ unsigned s_tk;
   // The chunks' partial sums (-dw, du), in sfold's space (used at other times).
   static_assert(2 * kFoldR + 1 >= kSW / 2, "spart must fit in sfold");
   auto spart = reinterpret_cast<float2(*)[32]>(&sfold[0][0]);
@@ -796,167 +827,155 @@ __global__ void __launch_bounds__(kSW * 32, 3)
   const int64_t nbg = int64_t(B) * G;
   const int nch = (T + kTT - 1) / kTT;
   const int nseg = (nch + kSW - 1) / kSW;
-  const unsigned nitems = unsigned(nbg * nseg);
   const BwdLayout lay = bwd_layout(ws, B, T, C);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  auto tile = [&](int buf, int i) { return dyn_tiles + ((buf * kSW + warp) * kNL + i) * kTile; };
-  // Lane 0 of each warp loads its own chunk of an item (no-op past the end of the sequence).
-  auto issue = [&](int buf, unsigned tk) {
-    const SegItem it = seg_item(tk, nbg, nseg, G);
-    const int ch = it.seg * kSW + warp;
-    if (ch < nch) {
-      uint64_t* bar = &bars[buf][warp];
-      mbar_arrive_expect_tx(bar, uint32_t(kNL) * kTile * sizeof(float));
-      for (int i = 0; i < kNL; ++i) tma_load_3d(tile(buf, i), &in_maps.m[i], bar, it.g << 5, ch * kTT, it.b);
-    }
-  };
-
+  if (threadIdx.x == 0) s_tk = atomicAdd(lay.rticket, 1u);
+  __syncthreads();
+  const unsigned tk = s_tk;
+  const int back = int(tk / nbg);  // segments from the end
+  const int seg = nseg - 1 - back;
+  const int64_t bg = int64_t(tk) - int64_t(back) * nbg;
+  const int b = int(bg / G);
+  const int g = int(bg - int64_t(b) * G);
+  const int c = (g << 5) + lane;
+  const bool valid = c < C;
+  const int ch = seg * kSW + warp;
+  const bool live = ch < nch;
+  const int t0 = ch * kTT;
+  const int64_t item0 = bg * nseg;
+  const int64_t item = item0 + seg;
+  float* tiles = dyn_tiles + warp * kNL * kTile;
+  float* K = tiles + lane;
+  float* V = tiles + kTile + lane;
+  float* R = tiles + 2 * kTile + lane;
+  float* DY = tiles + (kNL - 1) * kTile + lane;
+  uint64_t* bar = &bars[warp];
   if (lane == 0) {
-    mbar_init(&bars[0][warp], 1);
-    mbar_init(&bars[1][warp], 1);
+    mbar_init(bar, 1);
     mbar_fence_init();
+    if (live) {
+      mbar_arrive_expect_tx(bar, uint32_t(kNL) * kTile * sizeof(float));
+      for (int i = 0; i < kNL; ++i) tma_load_3d(tiles + i * kTile, &in_maps.m[i], bar, g << 5, t0, b);
+    }
   }
-  if (threadIdx.x == 0) {
-    s_tk[0] = atomicAdd(lay.rticket, 1u);
-    s_tk[1] = atomicAdd(lay.rticket, 1u);
+  __syncwarp();
+  const float4 ck = (live && valid) ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
+                                    : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
+  // The log2-scale of the state entering the next chunk (its checkpoint), see below.
+  const float2 nsc = (ch + 1 < nch && valid)
+                         ? *reinterpret_cast<const float2*>(
+                               &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z)
+                         : make_float2(0.f, 0.f);
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
+  const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+  const int rb = window_tokens(cp.w2, 128.f);
+  // The fold's inputs (step 2) are usually published long before they are needed: read
+  // their flags now (relaxed, not waited for) and only wait after pass 1 if one was not.
+  const int jc = min(nseg, seg + kFoldR + 1);
+  const int mfold = jc - 1 - seg;  // maps to apply
+  unsigned fearly = 0;
+  if (warp == kSW - 1) {
+    if (lane < mfold) fearly = ld_relaxed(&lay.rflags[item0 + seg + 1 + lane]);
+    if (lane == 31 && jc < nseg) fearly = ld_relaxed(&lay.rflags[item0 + jc]);
+  }
+
+  // ---- 1. forward recomputation and the chunk's reverse map ----
+  ChunkFactors f;
+  RevAgg A = rev_identity();
+  ChanState s;
+  s.a = ck.x;
+  s.b = ck.y;
+  s.Q = ck.z;
+  s.pl = ck.w;
+  if (live) {
+    mbar_wait(bar, 0, err);
+    __syncwarp();
+    A = fast ? chunk_forward_rb<GATE, DR, true>(s, cp, rb, K, V, R, DY, f)
+             : chunk_forward_rb<GATE, DR, false>(s, cp, rb, K, V, R, DY, f);
+  }
+  // The carry at this chunk's end comes scaled by the state entering the next chunk (its
+  // checkpoint); this chunk's own sums are scaled by its recomputed final state. Both are
+  // the same state reached by different orders of rounding: rescale by the exact ratio of
+  // the two scales (beta~ = beta 2^P) so the reverse sums stay consistent. The factor is
+  // folded into the chunk's map (E) for the chunks before it.
+  const float rme = (ch + 1 < nch) ? ex2(fminf((s.Q - nsc.x) + (s.pl - nsc.y), 64.f)) : 1.f;
+  A.E *= rme;
+  put_agg(&sagg[warp][lane][0], A);
+  __syncthreads();
+
+  // ---- 2. the segment's map; the carry at its end ----
+  if (warp == 0 && seg > 0) {  // the segment's map, for the segments before it
+    RevAgg M = get_agg(sagg[kSW - 1][lane][0], sagg[kSW - 1][lane][1]);
+#pragma unroll
+    for (int i = kSW - 2; i >= 0; --i) M = rev_compose(get_agg(sagg[i][lane][0], sagg[i][lane][1]), M);
+    put_agg(&lay.rmap[(item * 32 + lane) * 2], M);
+    warp_publish(&lay.rflags[item], 1u);
+  }
+  if (warp == kSW - 1) {
+    const int m = mfold;
+    const unsigned want = lane < m ? 1u : ((lane == 31 && jc < nseg) ? 2u : 0u);
+    // Each lane completes the acquire of its own flag before the warp barrier; the barrier
+    // then orders every lane's fetch below after all of them.
+    fence_acquire();
+    bool ok = true;
+    if (!__all_sync(0xffffffffu, fearly >= want)) {
+      unsigned fl = 1;
+      if (want != 0 && fearly < want)
+        fl = wait_flag(lane < m ? &lay.rflags[item0 + seg + 1 + lane] : &lay.rflags[item0 + jc],
+                       want, kWaitLimitNs, err);
+      ok = __all_sync(0xffffffffu, fl != 0);
+    }
+    RevCarry X{0.f, 0.f, 0.f, 0.f};
+    if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
+      // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
+      for (int l = 0; l < 2 * m; ++l)  // map of segment seg + 1 + l / 2, half l % 2
+        sfold[l][lane] = __ldcg(&lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
+      if (jc < nseg) {
+        const float4 q = __ldcg(&lay.carry[(item0 + jc) * 32 + lane]);
+        X = RevCarry{q.x, q.y, q.z, q.w};
+      }
+      __syncwarp();
+      for (int l = m - 1; l >= 0; --l)
+        X = rev_apply(get_agg(sfold[2 * l][lane], sfold[2 * l + 1][lane]), X);
+    }
+    sxe[lane] = make_float4(X.b, X.g, X.bd, X.gd);
   }
   __syncthreads();
-  unsigned tk = s_tk[0], tk_next = s_tk[1];
-  __syncthreads();  // (s_tk is rewritten in the loop)
-  if (tk < nitems && lane == 0) issue(0, tk);
-  uint32_t phase = 0;  // bit buf: parity of this warp's next wait on buffer buf
-  int buf = 0;
 
-  while (tk < nitems) {
-    // The next item's tiles into the other buffer, once this warp's stores of the item
-    // before have read it; and the ticket after the next.
-    if (lane == 0) {
-      tma_store_wait_read<0>();
-      if (tk_next < nitems) issue(buf ^ 1, tk_next);
-    }
-    if (threadIdx.x == 0) s_tk[buf] = tk_next < nitems ? atomicAdd(lay.rticket, 1u) : nitems;
-
-    const SegItem it = seg_item(tk, nbg, nseg, G);
-    const int seg = it.seg, b = it.b, g = it.g;
-    const int c = (g << 5) + lane;
-    const bool valid = c < C;
-    const int ch = seg * kSW + warp;
-    const bool live = ch < nch;
-    const int t0 = ch * kTT;
-    const int64_t item0 = it.bg * nseg;
-    const int64_t item = item0 + seg;
-    float* K = tile(buf, 0) + lane;
-    float* V = tile(buf, 1) + lane;
-    float* R = tile(buf, 2) + lane;
-    const float* DY = tile(buf, kNL - 1) + lane;
-    const float4 ck = (live && valid) ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
-                                      : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
-    // The log2-scale of the state entering the next chunk (its checkpoint), see below.
-    const float2 nsc = (ch + 1 < nch && valid)
-                           ? *reinterpret_cast<const float2*>(
-                                 &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z)
-                           : make_float2(0.f, 0.f);
-    const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
-    const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
-    const int rb = window_tokens(cp.w2, 128.f);
-
-    // ---- 1. forward recomputation and the chunk's reverse map ----
-    ChunkFactors f;
-    RevAgg A = rev_identity();
-    ChanState s;
-    s.a = ck.x;
-    s.b = ck.y;
-    s.Q = ck.z;
-    s.pl = ck.w;
-    if (live) {
-      mbar_wait(&bars[buf][warp], (phase >> buf) & 1u, err);
-      phase ^= 1u << buf;
-      __syncwarp();
-      A = fast ? chunk_forward_rb<GATE, DR, true>(s, cp, rb, K, V, R, DY, f)
-               : chunk_forward_rb<GATE, DR, false>(s, cp, rb, K, V, R, DY, f);
-    }
-    // The carry at this chunk's end comes scaled by the state entering the next chunk (its
-    // checkpoint); this chunk's own sums are scaled by its recomputed final state. Both are
-    // the same state reached by different orders of rounding: rescale by the exact ratio
-    // of the two scales (beta~ = beta 2^P) so the reverse sums stay consistent. The factor
-    // is folded into the chunk's map (E) for the chunks before it.
-    const float rme = (ch + 1 < nch) ? ex2(fminf((s.Q - nsc.x) + (s.pl - nsc.y), 64.f)) : 1.f;
-    A.E *= rme;
-    put_agg(&sagg[warp][lane][0], A);
-    __syncthreads();
-
-    // ---- 2. the segment's map; the carry at its end ----
-    if (warp == 0 && seg > 0) {  // the segment's map, for the segments before it
-      RevAgg M = get_agg(sagg[kSW - 1][lane][0], sagg[kSW - 1][lane][1]);
-#pragma unroll
-      for (int i = kSW - 2; i >= 0; --i) M = rev_compose(get_agg(sagg[i][lane][0], sagg[i][lane][1]), M);
-      put_agg(&lay.rmap[(item * 32 + lane) * 2], M);
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release(&lay.rflags[item], 1u);
-    }
-    if (warp == kSW - 1) {
-      const int jc = min(nseg, seg + kFoldR + 1);
-      const int m = jc - 1 - seg;  // maps to apply
-      unsigned fl = 1;
-      if (lane < m) fl = wait_flag(&lay.rflags[item0 + seg + 1 + lane], 1u, kWaitLimitNs, err);
-      if (lane == 31 && jc < nseg) fl = wait_flag(&lay.rflags[item0 + jc], 2u, kWaitLimitNs, err);
-      const bool ok = __all_sync(0xffffffffu, fl != 0);
-      RevCarry X{0.f, 0.f, 0.f, 0.f};
-      if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
-        // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
-        for (int l = 0; l < 2 * m; ++l)  // map of segment seg + 1 + l / 2, half l % 2
-          sfold[l][lane] = __ldcg(&lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
-        if (jc < nseg) {
-          const float4 q = __ldcg(&lay.carry[(item0 + jc) * 32 + lane]);
-          X = RevCarry{q.x, q.y, q.z, q.w};
-        }
-        __syncwarp();
-        for (int l = m - 1; l >= 0; --l)
-          X = rev_apply(get_agg(sfold[2 * l][lane], sfold[2 * l + 1][lane]), X);
-      }
-      sxe[lane] = make_float4(X.b, X.g, X.bd, X.gd);
-    }
-    __syncthreads();
-
-    // ---- 3. carries, reverse over the chunks ----
-    const float4 xe = sxe[lane];
-    RevCarry X{xe.x, xe.y, xe.z, xe.w};
-    for (int i = kSW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
-    if (warp == 0 && seg > kFoldR) {  // segment seg - kFoldR - 1 starts from this carry
-      const RevCarry X0 = rev_apply(A, X);
-      lay.carry[item * 32 + lane] = make_float4(X0.b, X0.g, X0.bd, X0.gd);
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release(&lay.rflags[item], 2u);
-    }
-    float2 part = make_float2(0.f, 0.f);
-    if (live) {
-      part = chunk_reverse(f, RevCarry{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme}, K, V);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        for (int i = 0; i < (DR ? 3 : 2); ++i) tma_store_3d(&out_maps.m[i], tile(buf, i), g << 5, t0, b);
-        tma_store_commit();
-      }
-    }
-    spart[warp][lane] = part;
-    __syncthreads();
-    if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
-      float sw = 0.f, su = 0.f;
-#pragma unroll
-      for (int i = 0; i < kSW; ++i) {
-        sw += spart[i][lane].x;
-        su += spart[i][lane].y;
-      }
-      lay.pdw[(int64_t(b) * nseg + seg) * C + c] = sw;
-      lay.pdu[(int64_t(b) * nseg + seg) * C + c] = su;
-    }
-    tk = tk_next;
-    tk_next = s_tk[buf];
-    buf ^= 1;
+  // ---- 3. carries, reverse over the chunks ----
+  const float4 xe = sxe[lane];
+  RevCarry X{xe.x, xe.y, xe.z, xe.w};
+  for (int i = kSW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
+  if (warp == 0 && seg > kFoldR) {  // segment seg - kFoldR - 1 starts from this carry
+    const RevCarry X0 = rev_apply(A, X);
+    lay.carry[item * 32 + lane] = make_float4(X0.b, X0.g, X0.bd, X0.gd);
+    warp_publish(&lay.rflags[item], 2u);
   }
-  if (lane == 0) tma_store_wait_all();
+  float2 part = make_float2(0.f, 0.f);
+  if (live) {
+    part = chunk_reverse(f, RevCarry{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme}, K, V, DY);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      for (int i = 0; i < (DR ? 3 : 2); ++i) tma_store_3d(&out_maps.m[i], tiles + i * kTile, g << 5, t0, b);
+      tma_store_commit();
+    }
+    __syncwarp();
+  }
+  spart[warp][lane] = part;  // (sfold's last reader, the fold, ended before the barrier above)
+  __syncthreads();
+  if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
+    float sw = 0.f, su = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSW; ++i) {
+      sw += spart[i][lane].x;
+      su += spart[i][lane].y;
+    }
+    lay.pdw[(int64_t(b) * nseg + seg) * C + c] = sw;
+    lay.pdu[(int64_t(b) * nseg + seg) * C + c] = su;
+  }
+  if (live && lane == 0) tma_store_wait_read<0>();  // the tiles stay until the stores read them
+  __syncwarp();
 }
 
 // ---- 3. reduction over batch rows and segments, fixed order -------------------------------
@@ -1012,19 +1031,12 @@ template <bool GATE, bool DR>
 int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, int64_t nitems,
                cudaStream_t stream) {
   auto kern = wkv_bwd_seg_kernel<GATE, DR>;
-  const size_t smem = 2 * size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
+  const size_t smem = size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return WKV_ERR_CUDA;
-  // Persistent: as many CTAs as fit at once (never more than there are items).
-  int dev = 0, sms = 0, per_sm = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSW * 32, smem) != cudaSuccess)
-    return WKV_ERR_CUDA;
-  const int64_t grid = std::min<int64_t>(nitems, int64_t(std::max(1, per_sm)) * sms);
-  kern<<<unsigned(grid), kSW * 32, smem, stream>>>(in, out, int(a.B), int(a.T), int(a.C), a.w,
-                                                    a.u, a.ws, a.err);
+  kern<<<unsigned(nitems), kSW * 32, smem, stream>>>(in, out, int(a.B), int(a.T), int(a.C), a.w,
+                                                      a.u, a.ws, a.err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -1050,7 +1062,9 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     if (nitems >= (int64_t(1) << 31)) return WKV_ERR_UNSUPPORTED;
     if (cudaMemsetAsync(a.ws, 0, bwd_flag_bytes(a.B, a.T, a.C), stream) != cudaSuccess)
       return WKV_ERR_CUDA;
-    wkv_bwd_ckpt_seg_kernel<<<unsigned(nitems), kSW * 32, 0, stream>>>(
+    const int64_t nch = (a.T + kTT - 1) / kTT;
+    const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
+    wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
         ck, int(a.B), int(a.T), int(a.C), a.w, a.ws, a.err);
     if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     if (a.r)

@@ -163,9 +163,7 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
                                        : agg_empty();
     } else {
       lay.agg[item * 32 + lane] = make_float4(A.a, A.b, A.ph, A.pl);
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release(&lay.flags[item], 1u);
+      warp_publish(&lay.flags[item], 1u);
       // Walk back: acc covers the segments between j and seg (exclusive), all full.
       Agg acc = agg_empty();
       int covered = 0;
@@ -204,9 +202,7 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
     const Agg incl = combine(carry, A, float(seg_len), cp.w2);
     if (!(withhold_seg0 && seg == 0)) {
       lay.incl[item * 32 + lane] = make_float4(incl.a, incl.b, incl.ph, incl.pl);
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release(&lay.flags[item], 2u);
+      warp_publish(&lay.flags[item], 2u);
     }
     scarry[lane] = make_float4(carry.a, carry.b, carry.ph, carry.pl);
   }
