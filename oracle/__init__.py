@@ -8,7 +8,8 @@ Two parts:
 
 * ``wkv_oracle.c`` (built into ``libwkv_oracle.so`` by :func:`build`), plain C in
   double precision: the O(T^2) parallel form, the unstabilised recurrence, the decode
-  step and the analytic backward;
+  step, the analytic backward and the backward through an entering and leaving state
+  (the recurrence's adjoint);
 * a few NumPy routines for tiny inputs that restate the operator through other
   routes: a causal softmax over logits (the operator as attention with
   query-independent weights), and one inference step written from the single-token
@@ -53,8 +54,9 @@ def _load():
         lib.oracle_wkv_recurrent.argtypes = [I, I, I] + [P] * 10
         lib.oracle_wkv_decode.argtypes = [I, I, I] + [P] * 8
         lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 13
+        lib.oracle_wkv_backward_state.argtypes = [I, I, I] + [P] * 19
         for f in (lib.oracle_wkv_direct, lib.oracle_wkv_recurrent, lib.oracle_wkv_decode,
-                  lib.oracle_wkv_backward):
+                  lib.oracle_wkv_backward, lib.oracle_wkv_backward_state):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -125,6 +127,27 @@ def wkv_backward(w, u, k, v, r, dy):
                                        _ptr(dy), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
                                        _ptr(dr), _ptr(dwa), _ptr(dua)))
     return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dw_abs": dwa, "du_abs": dua}
+
+
+def wkv_backward_state(w, u, k, v, r, dy, A0=None, B0=None, gA=None, gB=None):
+    """Gradients of sum(dy * y) + sum(gA * A_T) + sum(gB * B_T) for the forward from the
+    true initial state (A0, B0) [B, C] (None: empty), by the step-by-step adjoint of the
+    recurrence. Returns dict dk, dv, dw, du, dr (None if r is None), dA0, dB0 [B, C], and
+    dw_abs, du_abs: the same sums run on absolute values."""
+    w, u, k, v, r, dy, A0, B0, gA, gB = map(_f64, (w, u, k, v, r, dy, A0, B0, gA, gB))
+    B, T, C = k.shape
+    dk = np.empty((B, T, C))
+    dv = np.empty((B, T, C))
+    dr = np.empty((B, T, C)) if r is not None else None
+    dw, du, dwa, dua = (np.empty(C) for _ in range(4))
+    dA0 = np.empty((B, C))
+    dB0 = np.empty((B, C))
+    _check(_load().oracle_wkv_backward_state(
+        B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(dy), _ptr(A0), _ptr(B0),
+        _ptr(gA), _ptr(gB), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du), _ptr(dr), _ptr(dA0),
+        _ptr(dB0), _ptr(dwa), _ptr(dua)))
+    return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dA0": dA0, "dB0": dB0,
+            "dw_abs": dwa, "du_abs": dua}
 
 
 def state_from_scaled(a, b, p):

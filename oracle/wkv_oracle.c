@@ -212,3 +212,104 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
     free(D);
     return 0;
 }
+
+/*
+ * O5: gradients of the stateful forward (the backward through a state that enters and
+ * leaves, as when a long sequence is trained in consecutive pieces), by reverse-mode
+ * differentiation of the recurrence of [notes] "一句话总结" / "关键设计 2", written as
+ * its adjoint step by step. For 0-based t, with (A_{-1}, B_{-1}) = (A0, B0):
+ *   D_t   = B_{t-1} + e^{u+k_t},   wkv_t = (A_{t-1} + e^{u+k_t} v_t) / D_t,
+ *   y_t   = sigmoid(r_t) wkv_t,
+ *   A_t   = e^{-w} A_{t-1} + e^{k_t} v_t,   B_t = e^{-w} B_{t-1} + e^{k_t},
+ * and the loss L = sum_t dy_t y_t + gA A_{T-1} + gB B_{T-1} (gA, gB: the gradients of a
+ * later loss with respect to the final numerator and denominator). The adjoints
+ * Abar_t = dL/dA_t, Bbar_t = dL/dB_t run backward from (gA, gB):
+ *   g_t = dy_t sigmoid(r_t),
+ *   Abar_{t-1} = e^{-w} Abar_t + g_t / D_t,
+ *   Bbar_{t-1} = e^{-w} Bbar_t - g_t wkv_t / D_t,
+ *   dv_t = e^{k_t} Abar_t + g_t e^{u+k_t} / D_t,
+ *   dk_t = e^{k_t} (v_t Abar_t + Bbar_t) + g_t e^{u+k_t} (v_t - wkv_t) / D_t,
+ *   dw  -= e^{-w} (A_{t-1} Abar_t + B_{t-1} Bbar_t),
+ *   du  += g_t e^{u+k_t} (v_t - wkv_t) / D_t,
+ *   dr_t = dy_t wkv_t sigmoid(r_t) (1 - sigmoid(r_t)),
+ * and finally dA0 = Abar_{-1}, dB0 = Bbar_{-1}.
+ * A0, B0, gA, gB, dA0, dB0 are [B*C] and may be NULL (zero state / zero gradient / not
+ * wanted). dw_abs, du_abs (may be NULL) receive the same sums run on absolute values
+ * (|v|, |g|, |A0|, |gA|, |gB| in place of v, g, A0, gA, gB): the scale against which a
+ * float evaluation of dw and du is judged.
+ */
+int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
+                              const double *u, const double *k, const double *v,
+                              const double *r, const double *dy, const double *A0,
+                              const double *B0, const double *gA, const double *gB,
+                              double *dk, double *dv, double *dw, double *du, double *dr,
+                              double *dA0, double *dB0, double *dw_abs, double *du_abs)
+{
+    if (B < 0 || T < 0 || C < 0 || !w || !u || !dw || !du) return -1;
+    if (T > 0 && (!k || !v || !dy || !dk || !dv)) return -1;
+    size_t n = (size_t)(T > 0 ? T : 1) + 1;
+    /* Aprev[t] = A_{t-1} (index 0 holds the initial state), likewise the others */
+    double *Aprev = (double *)malloc(sizeof(double) * n);
+    double *Bprev = (double *)malloc(sizeof(double) * n);
+    double *Aabs = (double *)malloc(sizeof(double) * n);
+    double *D = (double *)malloc(sizeof(double) * n);
+    double *wkv = (double *)malloc(sizeof(double) * n);
+    if (!Aprev || !Bprev || !Aabs || !D || !wkv) {
+        free(Aprev); free(Bprev); free(Aabs); free(D); free(wkv);
+        return -1;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        dw[c] = 0.0;
+        du[c] = 0.0;
+        if (dw_abs) dw_abs[c] = 0.0;
+        if (du_abs) du_abs[c] = 0.0;
+    }
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t c = 0; c < C; ++c) {
+            const int64_t sc = b * C + c;
+            const double keep = exp(-w[c]);
+            double A = A0 ? A0[sc] : 0.0, Bd = B0 ? B0[sc] : 0.0, Aa = fabs(A);
+            for (int64_t t = 0; t < T; ++t) {                /* forward, keeping the past */
+                double kt = k[AT(b, t, c)], vt = v[AT(b, t, c)];
+                double bonus = exp(u[c] + kt);
+                Aprev[t] = A;
+                Bprev[t] = Bd;
+                Aabs[t] = Aa;
+                D[t] = Bd + bonus;
+                wkv[t] = (A + bonus * vt) / D[t];
+                A = keep * A + exp(kt) * vt;
+                Bd = keep * Bd + exp(kt);
+                Aa = keep * Aa + exp(kt) * fabs(vt);
+            }
+            double Abar = gA ? gA[sc] : 0.0, Bbar = gB ? gB[sc] : 0.0;
+            double Abar_a = fabs(Abar), Bbar_a = fabs(Bbar);
+            double dwc = 0.0, duc = 0.0, dwa = 0.0, dua = 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {           /* adjoint, last token first */
+                double kt = k[AT(b, t, c)], vt = v[AT(b, t, c)], dyt = dy[AT(b, t, c)];
+                double s = r ? sigm(r[AT(b, t, c)]) : 1.0;
+                double g = dyt * s;
+                double ek = exp(kt), bonus = exp(u[c] + kt);
+                /* Abar, Bbar here are dL/dA_t, dL/dB_t (this token's update feeds them) */
+                dv[AT(b, t, c)] = ek * Abar + g * bonus / D[t];
+                dk[AT(b, t, c)] = ek * (vt * Abar + Bbar) + g * bonus * (vt - wkv[t]) / D[t];
+                dwc -= keep * (Aprev[t] * Abar + Bprev[t] * Bbar);
+                duc += g * bonus * (vt - wkv[t]) / D[t];
+                dwa += keep * (Aabs[t] * Abar_a + Bprev[t] * Bbar_a);
+                dua += fabs(g) * bonus * (fabs(vt) + fabs(wkv[t])) / D[t];
+                if (r && dr) dr[AT(b, t, c)] = dyt * wkv[t] * s * (1.0 - s);
+                /* then step to dL/dA_{t-1}, dL/dB_{t-1} */
+                Abar = keep * Abar + g / D[t];
+                Bbar = keep * Bbar - g * wkv[t] / D[t];
+                Abar_a = keep * Abar_a + fabs(g) / D[t];
+                Bbar_a = keep * Bbar_a + fabs(g * wkv[t]) / D[t];
+            }
+            if (dA0) dA0[sc] = Abar;
+            if (dB0) dB0[sc] = Bbar;
+            dw[c] += dwc;
+            du[c] += duc;
+            if (dw_abs) dw_abs[c] += dwa;
+            if (du_abs) du_abs[c] += dua;
+        }
+    free(Aprev); free(Bprev); free(Aabs); free(D); free(wkv);
+    return 0;
+}

@@ -257,3 +257,79 @@ def test_golden_fixture_regression():
     y = oracle.wkv_direct(x.w, x.u, x.k, x.v, x.r)
     for b, t, c, val in rows:
         assert y[int(b), int(t), int(c)] == pytest.approx(float(val), rel=1e-13, abs=1e-15)
+
+
+def _loss_state(w, u, k, v, r, dy, A0, B0, gA, gB):
+    y, AT, BT = oracle.wkv_recurrent(w, u, k, v, r, A0, B0, want_state=True)
+    return float(np.sum(y * dy) + np.sum(gA * AT) + np.sum(gB * BT))
+
+
+def test_backward_state_matches_central_differences():
+    # The stateful backward (gradients through an entering and a leaving state) against
+    # central differences of sum(dy y) + gA A_T + gB B_T computed with the recurrence.
+    B, T, C = 2, 7, 3
+    w, u, k, v, r = _rand(B, T, C, 31)
+    g = np.random.Generator(np.random.PCG64(32))
+    dy = g.standard_normal((B, T, C))
+    A0 = g.standard_normal((B, C))
+    B0 = g.uniform(0.5, 2.0, (B, C))
+    gA = g.standard_normal((B, C))
+    gB = g.standard_normal((B, C))
+    res = oracle.wkv_backward_state(w, u, k, v, r, dy, A0, B0, gA, gB)
+    h = 1e-6
+    args = {"w": w, "u": u, "k": k, "v": v, "r": r, "A0": A0, "B0": B0}
+
+    def fd(name, idx):
+        a = dict(args)
+        p = a[name].copy(); p[idx] += h; a[name] = p
+        lp = _loss_state(a["w"], a["u"], a["k"], a["v"], a["r"], dy, a["A0"], a["B0"], gA, gB)
+        m = args[name].copy(); m[idx] -= h; a[name] = m
+        lm = _loss_state(a["w"], a["u"], a["k"], a["v"], a["r"], dy, a["A0"], a["B0"], gA, gB)
+        return (lp - lm) / (2 * h)
+
+    for name, key in (("k", "dk"), ("v", "dv"), ("r", "dr"), ("w", "dw"), ("u", "du"),
+                      ("A0", "dA0"), ("B0", "dB0")):
+        for idx in np.ndindex(args[name].shape):
+            assert fd(name, idx) == pytest.approx(res[key][idx], rel=1e-6, abs=1e-8), (name, idx)
+    assert np.all(res["dw_abs"] >= np.abs(res["dw"])) and np.all(res["du_abs"] >= np.abs(res["du"]))
+
+
+def test_backward_state_without_state_is_the_analytic_backward():
+    # Two independent derivations: the adjoint of the recurrence with empty state and
+    # zero final-state gradient, and the closed-form sums beta, gamma, betad, gammad.
+    w, u, k, v, r = _rand(3, 33, 4, 33)
+    dy = np.random.Generator(np.random.PCG64(34)).standard_normal((3, 33, 4))
+    a = oracle.wkv_backward(w, u, k, v, r, dy)
+    b = oracle.wkv_backward_state(w, u, k, v, r, dy)
+    for n in ("dk", "dv", "dr", "dw", "du"):
+        np.testing.assert_allclose(b[n], a[n], rtol=1e-12, atol=1e-13, err_msg=n)
+    np.testing.assert_allclose(b["dw_abs"], a["dw_abs"], rtol=1e-12, err_msg="dw_abs")
+    np.testing.assert_allclose(b["du_abs"], a["du_abs"], rtol=1e-12, err_msg="du_abs")
+
+
+def test_backward_state_chains_over_a_split_sequence():
+    # Training a sequence in two consecutive pieces: the second piece starts from the
+    # first's final state; its initial-state gradient is the first piece's final-state
+    # gradient. Together they must give the whole sequence's gradients.
+    B, T, C, T1 = 2, 30, 3, 11
+    w, u, k, v, r = _rand(B, T, C, 35)
+    g = np.random.Generator(np.random.PCG64(36))
+    dy = g.standard_normal((B, T, C))
+    A0 = g.standard_normal((B, C))
+    B0 = g.uniform(0.5, 2.0, (B, C))
+    gA = g.standard_normal((B, C))
+    gB = g.standard_normal((B, C))
+    whole = oracle.wkv_backward_state(w, u, k, v, r, dy, A0, B0, gA, gB)
+    _, Am, Bm = oracle.wkv_recurrent(w, u, k[:, :T1], v[:, :T1], r[:, :T1], A0, B0,
+                                     want_state=True)
+    second = oracle.wkv_backward_state(w, u, k[:, T1:], v[:, T1:], r[:, T1:], dy[:, T1:],
+                                       Am, Bm, gA, gB)
+    first = oracle.wkv_backward_state(w, u, k[:, :T1], v[:, :T1], r[:, :T1], dy[:, :T1],
+                                      A0, B0, second["dA0"], second["dB0"])
+    for n in ("dk", "dv", "dr"):
+        np.testing.assert_allclose(np.concatenate([first[n], second[n]], axis=1), whole[n],
+                                   rtol=1e-11, atol=1e-12, err_msg=n)
+    for n in ("dw", "du"):
+        np.testing.assert_allclose(first[n] + second[n], whole[n], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(first["dA0"], whole["dA0"], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(first["dB0"], whole["dB0"], rtol=1e-11, atol=1e-12)
