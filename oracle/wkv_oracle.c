@@ -234,16 +234,17 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
  *   dr_t = dy_t wkv_t sigmoid(r_t) (1 - sigmoid(r_t)),
  * and finally dA0 = Abar_{-1}, dB0 = Bbar_{-1}.
  * A0, B0, gA, gB, dA0, dB0 are [B*C] and may be NULL (zero state / zero gradient / not
- * wanted). dw_abs, du_abs (may be NULL) receive the same sums run on absolute values
- * (|v|, |g|, |A0|, |gA|, |gB| in place of v, g, A0, gA, gB): the scale against which a
- * float evaluation of dw and du is judged.
+ * wanted). dw_abs, du_abs, dA0_abs, dB0_abs (may be NULL) receive the same sums run on
+ * absolute values (|v|, |g|, |A0|, |gA|, |gB| in place of v, g, A0, gA, gB): the scale
+ * against which a float evaluation of these sums is judged.
  */
 int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
                               const double *u, const double *k, const double *v,
                               const double *r, const double *dy, const double *A0,
                               const double *B0, const double *gA, const double *gB,
                               double *dk, double *dv, double *dw, double *du, double *dr,
-                              double *dA0, double *dB0, double *dw_abs, double *du_abs)
+                              double *dA0, double *dB0, double *dw_abs, double *du_abs,
+                              double *dA0_abs, double *dB0_abs)
 {
     if (B < 0 || T < 0 || C < 0 || !w || !u || !dw || !du) return -1;
     if (T > 0 && (!k || !v || !dy || !dk || !dv)) return -1;
@@ -305,6 +306,8 @@ int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
             }
             if (dA0) dA0[sc] = Abar;
             if (dB0) dB0[sc] = Bbar;
+            if (dA0_abs) dA0_abs[sc] = Abar_a;
+            if (dB0_abs) dB0_abs[sc] = Bbar_a;
             dw[c] += dwc;
             du[c] += duc;
             if (dw_abs) dw_abs[c] += dwa;

@@ -292,6 +292,7 @@ def test_backward_state_matches_central_differences():
         for idx in np.ndindex(args[name].shape):
             assert fd(name, idx) == pytest.approx(res[key][idx], rel=1e-6, abs=1e-8), (name, idx)
     assert np.all(res["dw_abs"] >= np.abs(res["dw"])) and np.all(res["du_abs"] >= np.abs(res["du"]))
+    assert np.all(res["dA0_abs"] >= np.abs(res["dA0"])) and np.all(res["dB0_abs"] >= np.abs(res["dB0"]))
 
 
 def test_backward_state_without_state_is_the_analytic_backward():
