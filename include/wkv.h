@@ -173,6 +173,38 @@ WKV_API int wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const 
                          size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Backward of the stateful forward (wkv_forward_state with the same w, u, k, v, r and
+ * initial state), fp32: gradients of L = sum dy . y + L', where L' is a later loss that
+ * depends on the final state, as when a long sequence is trained in consecutive pieces.
+ * Defined, like wkv_backward, by the chain rule through the recurrence of the paper notes
+ * "RWKV - 把 RNN 重新带回 Transformer 时代的线性大模型", "一句话总结" (numerator and
+ * denominator decayed by e^{-w} and advanced by e^{k} v and e^{k}).
+ *   a0, b0, p0: the initial state given to the forward (fp32 [B, C], the representation of
+ *     wkv_forward_state: numerator a0 e^{p0}, denominator b0 e^{p0}); all NULL = the empty
+ *     state.
+ *   ga1, gb1:   dL'/da1 and dL'/db1 for the final state (a1, b1, p1) that the forward
+ *     returned, p1 its log-scale (fp32 [B, C]); all three NULL = no later loss. L' is
+ *     taken to depend on the state through its numerator a1 e^{p1} and denominator
+ *     b1 e^{p1} only (p is a scale, not information), so no gradient for p1 is needed.
+ *   da0, db0, dp0: dL/da0, dL/db0, dL/dp0 (fp32 [B, C], overwritten; dp0 = a0 da0 +
+ *     b0 db0); all NULL = not wanted. Passing one piece's (da0, db0, p0) as the previous
+ *     piece's (ga1, gb1, p1) chains the backward over consecutive pieces.
+ *   dk, dv, dr, dw, du, r, workspace (wkv_backward_workspace_bytes(B, T, C)): as
+ *     wkv_backward; dw includes the decay of the initial state and of the final state's
+ *     gradient.
+ * T == 0: dw, du are zeroed and the state's gradients pass through (the final state is
+ * the initial one). Each triple must be all NULL or all non-NULL (else
+ * WKV_ERR_INVALID_ARG). Deterministic, like wkv_backward.
+ */
+WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                               const float* k, const float* v, const float* r, const float* dy,
+                               const float* a0, const float* b0, const float* p0,
+                               const float* ga1, const float* gb1, const float* p1, float* dk,
+                               float* dv, float* dw, float* du, float* dr, float* da0,
+                               float* db0, float* dp0, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
  * Query and clear device-side errors. Synchronises `stream`, then returns WKV_ERR_TIMEOUT
  * if any kernel of this library on the current device gave up a bounded wait since the
  * last query (the outputs of that call are then undefined), WKV_ERR_CUDA if the stream

@@ -41,6 +41,16 @@ WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const fl
                                        float* dw, float* du, float* dr, void* workspace,
                                        size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Forces the plain (non-TMA) tile movement of wkv_backward_state; otherwise as it.
+ */
+WKV_API int wkv_testing_backward_state_plain(
+    int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+    const float* v, const float* r, const float* dy, const float* a0, const float* b0,
+    const float* p0, const float* ga1, const float* gb1, const float* p1, float* dk, float* dv,
+    float* dw, float* du, float* dr, float* da0, float* db0, float* dp0, void* workspace,
+    size_t workspace_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

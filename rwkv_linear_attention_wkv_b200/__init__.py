@@ -12,8 +12,8 @@ import ctypes
 import os
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
-           "wkv_backward", "wkv_backward_workspace_bytes", "wkv_stream_status",
-           "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
+           "wkv_backward", "wkv_backward_state", "wkv_backward_workspace_bytes",
+           "wkv_stream_status", "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
 
@@ -38,6 +38,9 @@ _SIGS = {
     "wkv_backward": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int),
     "wkv_testing_backward_plain": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P],
                                    ctypes.c_int),
+    "wkv_backward_state": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "wkv_testing_backward_state_plain": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
+                                         ctypes.c_int),
     "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
     "wkv_testing_forward_plain": ([_I, _I, _I] + [_P] * 6 + [ctypes.c_int, _P], ctypes.c_int),
 }
@@ -221,6 +224,58 @@ def wkv_backward(w, u, k, v, r, dy, want_dr=True, workspace=None, out=None, stre
         raise ValueError(f"workspace must be a CUDA tensor of at least {nbytes} bytes")
     _call(_entry, B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(dy),
           _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dw"]), _ptr(out["du"]), _ptr(out["dr"]),
+          _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    return out
+
+
+def wkv_backward_state(w, u, k, v, r, dy, state=None, grad_state=None, want_dr=True,
+                       workspace=None, out=None, stream=None, _entry="wkv_backward_state"):
+    """fp32 gradients for y, (a1, b1, p1) = wkv_forward_state(w, u, k, v, r, state).
+
+    `state` = (a0, b0, p0) or None (empty); `grad_state` = (ga1, gb1, p1): the gradients
+    of a later loss with respect to the final state's a1, b1, and that state's p1; or None.
+    Returns the dict of wkv_backward plus da0, db0, dp0 (B, C). Chaining: pass a piece's
+    (da0, db0, p0) as the previous piece's grad_state.
+    """
+    torch = _torch()
+    f32 = torch.float32
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    _need(k, "k", f32)
+    for n, t in (("v", v), ("dy", dy)):
+        _need(t, n, f32, (B, T, C))
+    if r is not None:
+        _need(r, "r", f32, (B, T, C))
+    _need(w, "w", f32, (C,))
+    _need(u, "u", f32, (C,))
+    st = tuple(state) if state is not None else (None, None, None)
+    gs = tuple(grad_state) if grad_state is not None else (None, None, None)
+    for n, t in zip(("a0", "b0", "p0", "ga1", "gb1", "p1"), st + gs):
+        if t is not None:
+            _need(t, n, f32, (B, C))
+    out = dict(out or {})
+    dev = k.device
+    for n, shape in (("dk", (B, T, C)), ("dv", (B, T, C)), ("dw", (C,)), ("du", (C,)),
+                     ("da0", (B, C)), ("db0", (B, C)), ("dp0", (B, C))):
+        if out.get(n) is None:
+            out[n] = torch.empty(shape, dtype=f32, device=dev)
+        _need(out[n], n, f32, shape)
+    if r is not None and want_dr:
+        if out.get("dr") is None:
+            out["dr"] = torch.empty((B, T, C), dtype=f32, device=dev)
+        _need(out["dr"], "dr", f32, (B, T, C))
+    else:
+        out["dr"] = None
+    nbytes = wkv_backward_workspace_bytes(B, T, C)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA tensor of at least {nbytes} bytes")
+    _call(_entry, B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(dy),
+          *(_ptr(t) for t in st + gs),
+          _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dw"]), _ptr(out["du"]), _ptr(out["dr"]),
+          _ptr(out["da0"]), _ptr(out["db0"]), _ptr(out["dp0"]),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return out
 

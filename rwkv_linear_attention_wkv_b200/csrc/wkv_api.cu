@@ -123,22 +123,52 @@ static int forward_impl(int64_t B, int64_t T, int64_t C, const float* w, const f
   return launch_fwd_stream(a, bf16, /*force_plain=*/T == 0, stream);
 }
 
+// The state arguments of wkv_backward_state (all NULL for wkv_backward).
+struct StateArgs {
+  const float* a0 = nullptr;
+  const float* b0 = nullptr;
+  const float* p0 = nullptr;
+  const float* ga1 = nullptr;
+  const float* gb1 = nullptr;
+  const float* p1 = nullptr;
+  float* da0 = nullptr;
+  float* db0 = nullptr;
+  float* dp0 = nullptr;
+};
+
+static bool all_or_none(const void* x, const void* y, const void* z) {
+  return (x == nullptr) == (y == nullptr) && (x == nullptr) == (z == nullptr);
+}
+
 static int backward_impl(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
                          const float* k, const float* v, const float* r, const float* dy,
                          float* dk, float* dv, float* dw, float* du, float* dr, void* workspace,
-                         size_t workspace_bytes, bool force_plain, cudaStream_t stream) {
+                         size_t workspace_bytes, bool force_plain, cudaStream_t stream,
+                         const StateArgs& st = StateArgs()) {
   if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
+  if (!all_or_none(st.a0, st.b0, st.p0) || !all_or_none(st.ga1, st.gb1, st.p1) ||
+      !all_or_none(st.da0, st.db0, st.dp0))
+    return WKV_ERR_INVALID_ARG;
   if (C == 0) return WKV_OK;
   if (!w || !u || !dw || !du) return WKV_ERR_INVALID_ARG;
   if (r == nullptr && dr != nullptr) return WKV_ERR_INVALID_ARG;
-  const void* ptrs[] = {w, u, k, v, r, dy, dk, dv, dw, du, dr};
+  const void* ptrs[] = {w,     u,     k,     v,      r,      dy,     dk,     dv,     dw, du,
+                        dr,    st.a0, st.b0, st.p0,  st.ga1, st.gb1, st.p1,  st.da0, st.db0,
+                        st.dp0};
   for (const void* q : ptrs)
     if (!aligned(q, 4)) return WKV_ERR_ALIGNMENT;
-  if (B == 0 || T == 0) {  // no tokens: zero gradients for the parameters
+  if (B == 0) return WKV_OK;
+  if (T == 0) {  // no tokens: zero gradients for the parameters; the state passes through
     if (cudaMemsetAsync(dw, 0, size_t(C) * sizeof(float), stream) != cudaSuccess ||
         cudaMemsetAsync(du, 0, size_t(C) * sizeof(float), stream) != cudaSuccess)
       return WKV_ERR_CUDA;
-    return WKV_OK;
+    if (st.da0 == nullptr) return WKV_OK;
+    if (B > INT64_MAX / C) return WKV_ERR_UNSUPPORTED;
+    BwdArgs a{B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, nullptr, nullptr};
+    a.a0 = st.a0; a.b0 = st.b0; a.p0 = st.p0;
+    a.ga1 = st.ga1; a.gb1 = st.gb1; a.p1 = st.p1;
+    a.da0 = st.da0; a.db0 = st.db0; a.dp0 = st.dp0;
+    return launch_backward_no_tokens(a, stream);
   }
   if (!k || !v || !dy || !dk || !dv) return WKV_ERR_INVALID_ARG;
   if (T >= (int64_t(1) << 31) || C >= (int64_t(1) << 31) || B >= (int64_t(1) << 31) ||
@@ -150,6 +180,9 @@ static int backward_impl(int64_t B, int64_t T, int64_t C, const float* w, const 
   unsigned* err = error_word();
   if (err == nullptr) return WKV_ERR_CUDA;
   BwdArgs a{B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace, err};
+  a.a0 = st.a0; a.b0 = st.b0; a.p0 = st.p0;
+  a.ga1 = st.ga1; a.gb1 = st.gb1; a.p1 = st.p1;
+  a.da0 = st.da0; a.db0 = st.db0; a.dp0 = st.dp0;
   return launch_backward(a, force_plain, stream);
 }
 
@@ -222,6 +255,21 @@ WKV_API int wkv_backward(int64_t B, int64_t T, int64_t C, const float* w, const 
                        workspace_bytes, false, stream);
 }
 
+WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                               const float* k, const float* v, const float* r, const float* dy,
+                               const float* a0, const float* b0, const float* p0,
+                               const float* ga1, const float* gb1, const float* p1, float* dk,
+                               float* dv, float* dw, float* du, float* dr, float* da0,
+                               float* db0, float* dp0, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
+  StateArgs st;
+  st.a0 = a0; st.b0 = b0; st.p0 = p0;
+  st.ga1 = ga1; st.gb1 = gb1; st.p1 = p1;
+  st.da0 = da0; st.db0 = db0; st.dp0 = dp0;
+  return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
+                       workspace_bytes, false, stream, st);
+}
+
 WKV_API int wkv_stream_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV_ERR_CUDA;
   unsigned* err = error_word();
@@ -285,6 +333,20 @@ WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const fl
                                        size_t workspace_bytes, cudaStream_t stream) {
   return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
                        workspace_bytes, true, stream);
+}
+
+WKV_API int wkv_testing_backward_state_plain(
+    int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+    const float* v, const float* r, const float* dy, const float* a0, const float* b0,
+    const float* p0, const float* ga1, const float* gb1, const float* p1, float* dk, float* dv,
+    float* dw, float* du, float* dr, float* da0, float* db0, float* dp0, void* workspace,
+    size_t workspace_bytes, cudaStream_t stream) {
+  StateArgs st;
+  st.a0 = a0; st.b0 = b0; st.p0 = p0;
+  st.ga1 = ga1; st.gb1 = gb1; st.p1 = p1;
+  st.da0 = da0; st.db0 = db0; st.dp0 = dp0;
+  return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
+                       workspace_bytes, true, stream, st);
 }
 
 }  // extern "C"

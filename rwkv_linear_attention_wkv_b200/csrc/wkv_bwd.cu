@@ -57,6 +57,7 @@ constexpr int kFoldR = 5;
 
 struct BwdLayout {
   float4* ckpt;      // [B, nch, C] forward state entering each chunk: (a, b, Q, pl)
+  float4* ckend;     // [B, C] forward state after the last token
   float* pdw;        // [B, nseg, C] per-segment partial sums of dw
   float* pdu;        // [B, nseg, C] per-segment partial sums of du
   unsigned* fticket;  // segment tickets of the checkpoint pass (forward chain)
@@ -95,6 +96,8 @@ __host__ __device__ inline BwdLayout bwd_layout(void* ws, int64_t B, int64_t T, 
   p += bwd_flag_bytes(B, T, C);
   L.ckpt = reinterpret_cast<float4*>(p);
   p += align256(size_t(B) * nch * C * sizeof(float4));
+  L.ckend = reinterpret_cast<float4*>(p);
+  p += align256(size_t(B) * C * sizeof(float4));
   L.pdw = reinterpret_cast<float*>(p);
   p += align256(size_t(B) * bwd_nseg(T) * C * sizeof(float));
   L.pdu = reinterpret_cast<float*>(p);
@@ -111,6 +114,7 @@ __host__ __device__ inline size_t bwd_bytes(int64_t B, int64_t T, int64_t C) {
   const int64_t nch = (T + kTT - 1) / kTT;
   const int64_t nitems = B * ((C + 31) / 32) * bwd_nseg(T);
   return bwd_flag_bytes(B, T, C) + align256(size_t(B) * nch * C * sizeof(float4)) +
+         align256(size_t(B) * C * sizeof(float4)) +
          2 * align256(size_t(B) * bwd_nseg(T) * C * sizeof(float)) +
          align256(size_t(nitems) * 32 * sizeof(float4)) +
          align256(size_t(nitems) * 32 * 2 * sizeof(float4)) +
@@ -203,6 +207,39 @@ struct TensorMaps4 {
   CUtensorMap m[4];
 };
 
+// Backward through a state (see BwdArgs): all NULL for the plain backward.
+struct StateIO {
+  const float* a0;
+  const float* b0;
+  const float* p0;
+  const float* ga1;
+  const float* gb1;
+  const float* p1;
+  float* da0;
+  float* db0;
+  float* dp0;
+};
+
+// The state entering the sequence: the given initial state, or the empty one.
+__device__ __forceinline__ ChanState initial_state(const StateIO& io, int64_t sidx, bool valid) {
+  return (io.a0 != nullptr && valid) ? load_state(io.a0[sidx], io.b0[sidx], io.p0[sidx])
+                                     : empty_state();
+}
+
+// The scaled reverse carry at the end of the sequence, from the gradients (ga1, gb1) of a
+// later loss with respect to the final state's a1, b1 (log-scale p1): beta = dL/dA_T =
+// ga1 e^{-p1}, gamma = -dL/dB_T = -gb1 e^{-p1}, both scaled by 2^P for the log2-scale P
+// = (Ph, Pl) of the state after the last token as this pass represents it.
+__device__ __forceinline__ float2 end_carry(const StateIO& io, int64_t sidx, bool valid,
+                                            float Ph, float Pl) {
+  if (io.ga1 == nullptr || !valid) return make_float2(0.f, 0.f);
+  const float p1 = io.p1[sidx];
+  const float qh = p1 * kLog2e;
+  const float ql = fmaf(p1, kLog2e, -qh);  // exact low part of the product
+  const float f = ex2(fminf((Ph - qh) + (Pl - ql), 126.f));
+  return make_float2(io.ga1[sidx] * f, -io.gb1[sidx] * f);
+}
+
 // ---- 1. checkpoints --------------------------------------------------------------------
 template <bool TMA>
 __global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_constant__ TensorMaps4 maps,
@@ -210,7 +247,8 @@ __global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_consta
                                                           const float* __restrict__ v,
                                                           int B, int T, int C,
                                                           const float* __restrict__ w,
-                                                          void* ws, unsigned* err) {
+                                                          const StateIO io, void* ws,
+                                                          unsigned* err) {
   constexpr int S = 3;
   constexpr int kTile = kTT * 32;
   __shared__ __align__(128) float tiles[S][2][kTile];  // per stage: k, v
@@ -236,7 +274,7 @@ __global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_consta
 
   ChanParams cp = chan_params(valid ? w[c] : 1.f, 0.f);
   const int rb = window_tokens(cp.w2, 128.f);
-  ChanState s = empty_state();
+  ChanState s = initial_state(io, int64_t(b) * C + c, valid);
   for (int ch = 0; ch < nch; ++ch) {
     const int st = ch % S;
     if (valid) lay.ckpt[(int64_t(b) * nch + ch) * C + c] = make_float4(s.a, s.b, s.Q, s.pl);
@@ -254,6 +292,7 @@ __global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_consta
     __syncwarp();
     if (ch + S < nch) issue(st, ch + S);
   }
+  if (valid) lay.ckend[int64_t(b) * C + c] = make_float4(s.a, s.b, s.Q, s.pl);
 }
 
 // Token weights for the time-parallel checkpoints and the recomputation that starts from
@@ -324,7 +363,7 @@ __device__ __forceinline__ Agg chunk_aggregate(const float* K, const float* V, i
 
 __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
     const __grid_constant__ TensorMaps4 maps, int B, int T, int C, const float* __restrict__ w,
-    void* ws, unsigned* err) {
+    const StateIO io, void* ws, unsigned* err) {
   constexpr int kTile = kTT * 32;
   constexpr int kSegC = kSW * kCK;  // chunks per checkpoint segment
   __shared__ __align__(128) float tiles[kSW][kCK][2][kTile];  // k, v of each warp's chunks
@@ -425,7 +464,7 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
                        kWaitLimitNs, err);
       ok = __all_sync(0xffffffffu, fl != 0);
     }
-    Agg X = agg_empty();
+    Agg X = j0 == 0 ? to_agg(initial_state(io, int64_t(b) * C + c, valid)) : agg_empty();
     if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
       // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
       for (int l = 0; l < m; ++l) sfold[l][lane] = __ldcg(&lay.fagg[(item0 + j0 + l) * 32 + lane]);
@@ -456,9 +495,11 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
       const int chq = ch0 + q2;
       if (chq < nch) {
         if (valid) ck[int64_t(chq) * C] = make_float4(X.a, X.b, X.ph, X.pl);
-        if (q2 + 1 < kCK) {
+        if (q2 + 1 < kCK || chq + 1 == nch) {
           const float4 a = sagg[warp * kCK + q2][lane];
-          X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kTT), cp.w2);
+          X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(min(kTT, T - chq * kTT)), cp.w2);
+          // after the last chunk: the state after the last token
+          if (chq + 1 == nch && valid) lay.ckend[int64_t(b) * C + c] = make_float4(X.a, X.b, X.ph, X.pl);
         }
       }
     }
@@ -477,7 +518,8 @@ __global__ void __launch_bounds__(32, 3) wkv_bwd_main_kernel(
     const __grid_constant__ TensorMaps4 in_maps, const __grid_constant__ TensorMaps4 out_maps,
     const float* __restrict__ k, const float* __restrict__ v, const float* __restrict__ r,
     const float* __restrict__ dy, float* dk, float* dv, float* dr, int B, int T, int C,
-    const float* __restrict__ w, const float* __restrict__ u, void* ws, unsigned* err) {
+    const float* __restrict__ w, const float* __restrict__ u, const StateIO io, void* ws,
+    unsigned* err) {
   constexpr int kTile = kTT * 32;
   extern __shared__ __align__(128) float smem[];
   // stage s2 holds tiles k, v, r (or dy), dy at smem + (4 s2 + slot) kTile
@@ -590,6 +632,13 @@ __global__ void __launch_bounds__(32, 3) wkv_bwd_main_kernel(
         j = 0;
       }
     }
+    if (it == 0) {  // the last chunk: the carry after the last token, from a later loss
+      float Ph = s.Q, Pl = s.pl;
+      if (j) decay_pair(s.Q, s.pl, float(j), cp.w2, Ph, Pl);  // mid-window: P after token T-1
+      const float2 e = end_carry(io, int64_t(b) * C + c, valid, Ph, Pl);
+      beta = e.x;
+      gamma = e.y;
+    }
     // Reverse over the chunk; dk, dv (dr) replace k, v (r) in shared memory.
 #pragma unroll 8
     for (int t = n - 1; t >= 0; --t) {
@@ -611,6 +660,16 @@ __global__ void __launch_bounds__(32, 3) wkv_bwd_main_kernel(
       gammad = e1 * (gammad + gamma);
       beta = fmaf(e1, beta, inj);
       gamma = fmaf(e1, gamma, inj * wk);
+    }
+    if (ch == 0) {  // the start of the sequence: the initial state's gradients
+      const float a0 = valid ? ck.x : 0.f, b0 = valid ? ck.y : 0.f;  // ck: the initial state
+      if (io.da0 != nullptr && valid) {
+        const int64_t sidx = int64_t(b) * C + c;
+        io.da0[sidx] = beta;
+        io.db0[sidx] = -gamma;
+        io.dp0[sidx] = fmaf(a0, beta, -b0 * gamma);
+      }
+      dw_acc = fmaf(a0, betad, fmaf(-b0, gammad, dw_acc));  // -dw_acc is stored below
     }
     if (ch % kSW == 0) {  // the segment's first chunk: its partial sums are complete
       if (valid) {
@@ -766,13 +825,16 @@ __device__ __forceinline__ RevAgg chunk_forward_rb(ChanState& s, const ChanParam
   return chunk_forward<GATE, DR, FASTOUT, 1>(s, cp, K, V, R, DY, f);
 }
 
-// Reverse over one chunk from the carry X at its end: dk, dv replace wkv (in K), v in shared
-// memory; returns the chunk's partial sums of -dw (.x) and du (.y).
+// Reverse over one chunk from the carry X after its last real token (position nvalid - 1;
+// TAIL: nvalid < kTT, the positions after it are skipped): dk, dv replace wkv (in K), v in
+// shared memory; returns the chunk's partial sums of -dw (.x) and du (.y).
+template <bool TAIL>
 __device__ __forceinline__ float2 chunk_reverse(const ChunkFactors& f, RevCarry X, float* K,
-                                                float* V, const float* CUR) {
+                                                float* V, const float* CUR, int nvalid) {
   float dw_acc = 0.f, du_acc = 0.f;
 #pragma unroll
   for (int t = kTT - 1; t >= 0; --t) {
+    if (TAIL && t >= nvalid) continue;
     const float vv = V[t * 32], wk = K[t * 32], cur = CUR[t * 32];
     const bool dom = (f.tok >> t) & 1u;
     const float e1 = dom ? f.fe[t] : 1.f;
@@ -808,8 +870,8 @@ template <bool GATE, bool DR>
 __global__ void __launch_bounds__(kSW * 32, 5)
     wkv_bwd_seg_kernel(const __grid_constant__ TensorMaps4 in_maps,
                        const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
-                       const float* __restrict__ w, const float* __restrict__ u, void* ws,
-                       unsigned* err) {
+                       const float* __restrict__ w, const float* __restrict__ u,
+                       const StateIO io, void* ws, unsigned* err) {
   constexpr int kTile = kTT * 32;
   constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
   // Dynamic: [kSW warps][kNL tiles][kTile] floats.
@@ -861,11 +923,15 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   __syncwarp();
   const float4 ck = (live && valid) ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
                                     : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
-  // The log2-scale of the state entering the next chunk (its checkpoint), see below.
-  const float2 nsc = (ch + 1 < nch && valid)
+  // The log2-scale of the state entering the next chunk (its checkpoint; after the last
+  // chunk, the state after the last token), see below.
+  const int64_t sidx = int64_t(b) * C + c;
+  const float2 nsc = (ch < nch && valid)
                          ? *reinterpret_cast<const float2*>(
-                               &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z)
+                               ch + 1 < nch ? &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z
+                                            : &lay.ckend[sidx].z)
                          : make_float2(0.f, 0.f);
+  const int nvalid = min(kTT, T - t0);  // real tokens of this chunk
   const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
   const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
   const int rb = window_tokens(cp.w2, 128.f);
@@ -890,15 +956,23 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   if (live) {
     mbar_wait(bar, 0, err);
     __syncwarp();
+    // Past the last token (zero-filled tiles): a weight of 2^{-huge} makes the positions
+    // inert (e1 = 1, e2 = 0: the state and the reverse sums pass through unchanged).
+    for (int t = nvalid; t < kTT; ++t) K[t * 32] = -1.0e30f;
     A = fast ? chunk_forward_rb<GATE, DR, true>(s, cp, rb, K, V, R, DY, f)
              : chunk_forward_rb<GATE, DR, false>(s, cp, rb, K, V, R, DY, f);
+    A.L = float(nvalid);  // the inert positions add no distance
   }
   // The carry at this chunk's end comes scaled by the state entering the next chunk (its
-  // checkpoint); this chunk's own sums are scaled by its recomputed final state. Both are
-  // the same state reached by different orders of rounding: rescale by the exact ratio of
-  // the two scales (beta~ = beta 2^P) so the reverse sums stay consistent. The factor is
-  // folded into the chunk's map (E) for the chunks before it.
-  const float rme = (ch + 1 < nch) ? ex2(fminf((s.Q - nsc.x) + (s.pl - nsc.y), 64.f)) : 1.f;
+  // checkpoint, or the state after the last token); this chunk's own sums are scaled by
+  // its recomputed state after its last real token. Both are the same state reached by
+  // different orders of rounding: rescale by the exact ratio of the two scales
+  // (beta~ = beta 2^P) so the reverse sums stay consistent. The factor is folded into the
+  // chunk's map (E) for the chunks before it. (Inert positions after the last token moved
+  // the frame on by (kTT - nvalid) w2: undone here.)
+  float Ph = s.Q, Pl = s.pl;
+  if (nvalid < kTT) decay_pair(s.Q, s.pl, float(nvalid - kTT), cp.w2, Ph, Pl);
+  const float rme = (live && valid) ? ex2(fminf((Ph - nsc.x) + (Pl - nsc.y), 64.f)) : 1.f;
   A.E *= rme;
   put_agg(&sagg[warp][lane][0], A);
   __syncthreads();
@@ -926,6 +1000,11 @@ __global__ void __launch_bounds__(kSW * 32, 5)
       ok = __all_sync(0xffffffffu, fl != 0);
     }
     RevCarry X{0.f, 0.f, 0.f, 0.f};
+    if (jc == nseg && io.ga1 != nullptr && valid) {  // the carry at the end of the sequence
+      const float4 q = lay.ckend[sidx];
+      const float2 e = end_carry(io, sidx, valid, q.z, q.w);
+      X = RevCarry{e.x, e.y, 0.f, 0.f};
+    }
     if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
       // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
       for (int l = 0; l < 2 * m; ++l)  // map of segment seg + 1 + l / 2, half l % 2
@@ -951,9 +1030,24 @@ __global__ void __launch_bounds__(kSW * 32, 5)
     lay.carry[item * 32 + lane] = make_float4(X0.b, X0.g, X0.bd, X0.gd);
     warp_publish(&lay.rflags[item], 2u);
   }
+  float dw_init = 0.f;  // the initial state's part of dw (first segment)
+  if (warp == 0 && seg == 0) {
+    // The carry at the start of the sequence is scaled by the initial state's own scale
+    // (the first checkpoint is that state as given): beta~ = e^{p0} dL/dA0 = dL/da0.
+    const RevCarry X0 = rev_apply(A, X);
+    const float a0 = ck.x, b0 = ck.y;
+    if (io.da0 != nullptr && valid) {
+      io.da0[sidx] = X0.b;
+      io.db0[sidx] = -X0.g;
+      io.dp0[sidx] = fmaf(a0, X0.b, -b0 * X0.g);
+    }
+    dw_init = -fmaf(a0, X0.bd, -b0 * X0.gd);
+  }
   float2 part = make_float2(0.f, 0.f);
   if (live) {
-    part = chunk_reverse(f, RevCarry{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme}, K, V, DY);
+    const RevCarry Xc{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme};
+    part = nvalid == kTT ? chunk_reverse<false>(f, Xc, K, V, DY, kTT)
+                         : chunk_reverse<true>(f, Xc, K, V, DY, nvalid);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
@@ -965,7 +1059,7 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   spart[warp][lane] = part;  // (sfold's last reader, the fold, ended before the barrier above)
   __syncthreads();
   if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
-    float sw = 0.f, su = 0.f;
+    float sw = dw_init, su = 0.f;
 #pragma unroll
     for (int i = 0; i < kSW; ++i) {
       sw += spart[i][lane].x;
@@ -1009,6 +1103,10 @@ __global__ void __launch_bounds__(32 * kRS) wkv_bwd_reduce_kernel(int B, int C, 
   }
 }
 
+StateIO state_io(const BwdArgs& a) {
+  return StateIO{a.a0, a.b0, a.p0, a.ga1, a.gb1, a.p1, a.da0, a.db0, a.dp0};
+}
+
 size_t bwd_main_smem() {
   return (4 * kMS + 6) * kTT * 32 * sizeof(float) + kMS * sizeof(uint64_t);
 }
@@ -1023,7 +1121,8 @@ int launch_main(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
     return WKV_ERR_CUDA;
   const int64_t grid = a.B * ((a.C + 31) / 32);
   kern<<<unsigned(grid), 32, smem, stream>>>(in, out, a.k, a.v, a.r, a.dy, a.dk, a.dv, a.dr,
-                                             int(a.B), int(a.T), int(a.C), a.w, a.u, a.ws, a.err);
+                                             int(a.B), int(a.T), int(a.C), a.w, a.u,
+                                             state_io(a), a.ws, a.err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -1036,7 +1135,7 @@ int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, 
       cudaSuccess)
     return WKV_ERR_CUDA;
   kern<<<unsigned(nitems), kSW * 32, smem, stream>>>(in, out, int(a.B), int(a.T), int(a.C), a.w,
-                                                      a.u, a.ws, a.err);
+                                                      a.u, state_io(a), a.ws, a.err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -1065,7 +1164,7 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     const int64_t nch = (a.T + kTT - 1) / kTT;
     const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
     wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
-        ck, int(a.B), int(a.T), int(a.C), a.w, a.ws, a.err);
+        ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err);
     if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     if (a.r)
       rc = a.dr ? launch_seg<true, true>(a, in, out, nitems, stream)
@@ -1074,7 +1173,8 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
       rc = launch_seg<false, false>(a, in, out, nitems, stream);
   } else {
     wkv_bwd_ckpt_kernel<TMA><<<unsigned(grid), 32, 0, stream>>>(ck, a.k, a.v, int(a.B), int(a.T),
-                                                                int(a.C), a.w, a.ws, a.err);
+                                                                int(a.C), a.w, state_io(a), a.ws,
+                                                                a.err);
     if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     if (a.r)
       rc = a.dr ? launch_main<TMA, true, true>(a, in, out, stream)
@@ -1091,6 +1191,31 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
 }  // namespace
 
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C) { return bwd_bytes(B, T, C); }
+
+namespace {
+// No tokens: the final state is the initial one, so dL/dA0 = dL/dA_T = ga1 e^{-p1} and
+// da0 = e^{p0} dL/dA0 (the same for b); dp0 = a0 da0 + b0 db0.
+__global__ void wkv_bwd_no_tokens_kernel(int64_t n, const StateIO io) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float a0 = io.a0 ? io.a0[i] : 0.f, b0 = io.a0 ? io.b0[i] : 0.f;
+  float da = 0.f, db = 0.f;
+  if (io.ga1 != nullptr && io.a0 != nullptr) {
+    const float f = ex2(fminf((io.p0[i] - io.p1[i]) * kLog2e, 126.f));
+    da = io.ga1[i] * f;
+    db = io.gb1[i] * f;
+  }
+  io.da0[i] = da;
+  io.db0[i] = db;
+  io.dp0[i] = fmaf(a0, da, b0 * db);
+}
+}  // namespace
+
+int launch_backward_no_tokens(const BwdArgs& a, cudaStream_t stream) {
+  const int64_t n = a.B * a.C;
+  wkv_bwd_no_tokens_kernel<<<unsigned((n + 255) / 256), 256, 0, stream>>>(n, state_io(a));
+  return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
 
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream) {
   auto al16 = [](const void* p) {

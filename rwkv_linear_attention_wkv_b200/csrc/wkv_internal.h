@@ -88,8 +88,22 @@ struct BwdArgs {
   float* dr;
   void* ws;
   unsigned* err;
+  // Backward through a state (all may be NULL): the initial state (a0, b0, p0) [B, C];
+  // the gradients (ga1, gb1) of a later loss with respect to the final state's a1, b1,
+  // whose log-scale is p1 [B, C]; and the outputs (da0, db0, dp0) [B, C].
+  const float* a0 = nullptr;
+  const float* b0 = nullptr;
+  const float* p0 = nullptr;
+  const float* ga1 = nullptr;
+  const float* gb1 = nullptr;
+  const float* p1 = nullptr;
+  float* da0 = nullptr;
+  float* db0 = nullptr;
+  float* dp0 = nullptr;
 };
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);
+// T == 0 with the state's gradients wanted: they pass straight through.
+int launch_backward_no_tokens(const BwdArgs& a, cudaStream_t stream);
 
 }  // namespace wkv

@@ -81,15 +81,38 @@ def test_decode_and_backward_argument_checks(W):
 
 def test_backward_workspace_size(W):
     # Chain flags (16 bytes of tickets, then two words per segment item), the forward state
-    # (a, b, Q, pl) entering every 16-token chunk, per-segment partials of dw and du, and per
-    # segment item of 4 chunks and lane: its forward aggregate (1 float4), reverse map
-    # (2 float4) and reverse carry (1 float4).
+    # (a, b, Q, pl) entering every 16-token chunk and after the last token, per-segment
+    # partials of dw and du, and per segment item of 4 chunks and lane: its forward
+    # aggregate (1 float4), reverse map (2 float4) and reverse carry (1 float4).
     def a256(x):
         return (x + 255) // 256 * 256
     for B, T, C in ((16, 1024, 768), (1, 33, 5), (3, 1, 4096)):
         nch = (T + 15) // 16
         nseg = (nch + 3) // 4
         nitems = B * ((C + 31) // 32) * nseg
-        want = (a256(16 + 8 * nitems) + a256(B * nch * C * 16) + 2 * a256(B * nseg * C * 4)
-                + a256(nitems * 32 * 16) + a256(nitems * 32 * 32) + a256(nitems * 32 * 16))
+        want = (a256(16 + 8 * nitems) + a256(B * nch * C * 16) + a256(B * C * 16)
+                + 2 * a256(B * nseg * C * 4) + a256(nitems * 32 * 16) + a256(nitems * 32 * 32)
+                + a256(nitems * 32 * 16))
         assert W.wkv_backward_workspace_bytes(B, T, C) == want
+
+
+def test_backward_state_argument_checks(W):
+    ok = P(4096)
+    bs = W.lib.wkv_backward_state
+    need = W.wkv_backward_workspace_bytes(2, 64, 32)
+    base = [ok] * 6                      # w, u, k, v, r, dy
+    outs = [ok] * 5                      # dk, dv, dw, du, dr
+    full = [ok] * 3
+
+    def call(B, st, gs, ds, ws=ok, nb=need):
+        return bs(B, 64, 32, *base, *st, *gs, *outs, *ds, ws, nb, None)
+
+    none3 = [None] * 3
+    # each of the three triples must be all NULL or all non-NULL
+    assert call(2, [ok, None, ok], none3, none3) == 1
+    assert call(2, none3, [ok, ok, None], none3) == 1
+    assert call(2, none3, none3, [None, ok, ok]) == 1
+    assert call(2, full, full, full, nb=need - 1) == 1          # workspace too small
+    assert call(2, full, full, [ok, ok, P(4098)]) == 2          # dp0 not 4-byte aligned
+    assert call(-2, full, full, full) == 1
+    assert call(0, full, full, full) == 0                       # no batch rows: nothing
