@@ -399,7 +399,7 @@ def run_workload(args):
         n = x.B * x.T * x.C
         y = torch.empty_like(k)
         ms = _time_loop(lambda: W.wkv_forward(w, u, k, v, r, y=y), args.steps, args.warmup, stream)
-        line("train_169m", "forward fp32 16x1024x768 (chunked kernel)", ms, n, 16 * n)
+        line("train_169m", "forward fp32 16x1024x768 (streaming kernel)", ms, n, 16 * n)
         ws = torch.empty(W.wkv_backward_workspace_bytes(x.B, x.T, x.C), dtype=torch.uint8,
                          device=dev)
         out = {nm: torch.empty_like(k) for nm in ("dk", "dv", "dr")}
@@ -408,6 +408,21 @@ def run_workload(args):
         ms = _time_loop(lambda: W.wkv_backward(w, u, k, v, r, dy, workspace=ws, out=out),
                         args.steps, args.warmup, stream)
         line("train_169m", "backward fp32 16x1024x768 (dk, dv, dr, dw, du)", ms, n, 28 * n)
+        # the same through an entering and a leaving state (one piece of a longer sequence)
+        g = np.random.Generator(np.random.PCG64(1))
+        st = (d(g.standard_normal((x.B, x.C)).astype(np.float32)),
+              d(g.uniform(0.5, 2.0, (x.B, x.C)).astype(np.float32)),
+              d(g.normal(0.0, 2.0, (x.B, x.C)).astype(np.float32)))
+        _, st1 = W.wkv_forward_state(w, u, k, v, r, state=st)
+        gs = (d(g.standard_normal((x.B, x.C)).astype(np.float32)),
+              d(g.standard_normal((x.B, x.C)).astype(np.float32)), st1[2])
+        for nm in ("da0", "db0", "dp0"):
+            out[nm] = torch.empty((x.B, x.C), device=dev)
+        ms = _time_loop(lambda: W.wkv_backward_state(w, u, k, v, r, dy, state=st, grad_state=gs,
+                                                     workspace=ws, out=out),
+                        args.steps, args.warmup, stream)
+        line("train_169m", "backward_state fp32 16x1024x768 (with initial state and final-state "
+             "gradients)", ms, n, 28 * n + 36 * x.B * x.C)
     elif args.workload == "long_ctx":
         x = wkv_inputs.long_context(seed=0, T=args.seq or 32768)
         w, u, k, v, r = (d(a) for a in (x.w, x.u, x.k, x.v, x.r))
