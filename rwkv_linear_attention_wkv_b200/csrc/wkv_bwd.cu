@@ -410,14 +410,24 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
   const ChanParams cp = chan_params(valid ? w[c] : 1.f, 0.f);
   const int rb = window_tokens(cp.w2, 128.f);
 
-  // The fold's inputs (below) are usually published long before they are needed: read
-  // their flags now (relaxed, not waited for) and only wait later if one was not.
+  // The fold's inputs (below) are usually published before this segment starts: the last
+  // warp checks their flags now (one acquire load per lane, while the tiles load) and, if
+  // all are set, copies them into shared memory (cp.async) while the aggregates are
+  // formed; otherwise it waits for them after that.
   const int j0 = max(0, seg - kFoldF);
   const int mfold = seg - j0;  // aggregates to fold
-  unsigned fearly = 0;
+  const unsigned fwant = lane < mfold ? 1u : ((lane == 31 && j0 > 0) ? 2u : 0u);
+  bool fold_early = false;
   if (warp == kSW - 1) {
-    if (lane < mfold) fearly = ld_relaxed(&lay.fflags[item0 + j0 + lane]);
-    if (lane == 31 && j0 > 0) fearly = ld_relaxed(&lay.fflags[item0 + j0]);
+    const unsigned* flag = lane < mfold ? &lay.fflags[item0 + j0 + lane] : &lay.fflags[item0 + j0];
+    const unsigned fl = fwant != 0 ? ld_acquire(flag) : 0u;
+    fold_early = __all_sync(0xffffffffu, fl >= fwant);
+    __syncwarp();  // orders every lane's acquire before every lane's copies below
+    if (fold_early) {
+      for (int l = 0; l < mfold; ++l) cp_async_16(&sfold[l][lane], &lay.fagg[(item0 + j0 + l) * 32 + lane]);
+      if (j0 > 0 && valid) cp_async_16(&sin_[lane], &ck[int64_t(j0) * kSegC * C]);
+      cp_async_commit();
+    }
   }
 
   // ---- the chunks' aggregates from the empty state ----
@@ -452,32 +462,31 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
   // ---- the state entering the segment (last warp; the aggregate above does not wait) ----
   if (warp == kSW - 1) {
     const int m = mfold;
-    const unsigned want = lane < m ? 1u : ((lane == 31 && j0 > 0) ? 2u : 0u);
-    // Each lane completes the acquire of its own flag before the warp barrier; the barrier
-    // then orders every lane's fetch below after all of them.
-    fence_acquire();
     bool ok = true;
-    if (!__all_sync(0xffffffffu, fearly >= want)) {
-      unsigned fl = 1;
-      if (want != 0 && fearly < want)
-        fl = wait_flag(lane < m ? &lay.fflags[item0 + j0 + lane] : &lay.fflags[item0 + j0], want,
-                       kWaitLimitNs, err);
+    if (fold_early) {
+      cp_async_wait_all();
+    } else {  // wait for the flags not yet set, then fetch (L2 loads: L1 may be stale)
+      const unsigned* flag = lane < m ? &lay.fflags[item0 + j0 + lane] : &lay.fflags[item0 + j0];
+      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, kWaitLimitNs, err) : 1u;
       ok = __all_sync(0xffffffffu, fl != 0);
-    }
-    Agg X = j0 == 0 ? to_agg(initial_state(io, int64_t(b) * C + c, valid)) : agg_empty();
-    if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
-      // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
-      for (int l = 0; l < m; ++l) sfold[l][lane] = __ldcg(&lay.fagg[(item0 + j0 + l) * 32 + lane]);
-      if (j0 > 0 && valid) {
-        const float4 q = __ldcg(&ck[int64_t(j0) * kSegC * C]);
-        X = Agg{q.x, q.y, q.z, q.w};
+      __syncwarp();  // orders every lane's acquire before every lane's fetch below
+      if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
+        for (int l = 0; l < m; ++l) sfold[l][lane] = __ldcg(&lay.fagg[(item0 + j0 + l) * 32 + lane]);
+        if (j0 > 0 && valid) sin_[lane] = __ldcg(&ck[int64_t(j0) * kSegC * C]);
       }
-      __syncwarp();
+    }
+    __syncwarp();
+    Agg X = to_agg(initial_state(io, int64_t(b) * C + c, valid));
+    if (j0 > 0) {
+      const float4 q = sin_[lane];
+      X = (ok && valid) ? Agg{q.x, q.y, q.z, q.w} : agg_empty();
+    }
+    if (ok)
       for (int l = 0; l < m; ++l) {
         const float4 a = sfold[l][lane];
         X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kSegC * kTT), cp.w2);
       }
-    }
+    __syncwarp();
     sin_[lane] = make_float4(X.a, X.b, X.ph, X.pl);
   }
   __syncthreads();
@@ -935,14 +944,25 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
   const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
   const int rb = window_tokens(cp.w2, 128.f);
-  // The fold's inputs (step 2) are usually published long before they are needed: read
-  // their flags now (relaxed, not waited for) and only wait after pass 1 if one was not.
+  // The fold's inputs (step 2) are usually published before this segment starts: the last
+  // warp checks their flags now (one acquire load per lane, while the tiles load) and, if
+  // all are set, copies them into shared memory (cp.async) during the forward
+  // recomputation; otherwise it waits for them after that.
   const int jc = min(nseg, seg + kFoldR + 1);
   const int mfold = jc - 1 - seg;  // maps to apply
-  unsigned fearly = 0;
+  const unsigned fwant = lane < mfold ? 1u : ((lane == 31 && jc < nseg) ? 2u : 0u);
+  bool fold_early = false;
   if (warp == kSW - 1) {
-    if (lane < mfold) fearly = ld_relaxed(&lay.rflags[item0 + seg + 1 + lane]);
-    if (lane == 31 && jc < nseg) fearly = ld_relaxed(&lay.rflags[item0 + jc]);
+    const unsigned* flag = lane < mfold ? &lay.rflags[item0 + seg + 1 + lane] : &lay.rflags[item0 + jc];
+    const unsigned fl = fwant != 0 ? ld_acquire(flag) : 0u;
+    fold_early = __all_sync(0xffffffffu, fl >= fwant);
+    __syncwarp();  // orders every lane's acquire before every lane's copies below
+    if (fold_early) {
+      for (int l = 0; l < 2 * mfold; ++l)  // map of segment seg + 1 + l / 2, half l % 2
+        cp_async_16(&sfold[l][lane], &lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
+      if (jc < nseg) cp_async_16(&sfold[2 * mfold][lane], &lay.carry[(item0 + jc) * 32 + lane]);
+      cp_async_commit();
+    }
   }
 
   // ---- 1. forward recomputation and the chunk's reverse map ----
@@ -987,36 +1007,35 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   }
   if (warp == kSW - 1) {
     const int m = mfold;
-    const unsigned want = lane < m ? 1u : ((lane == 31 && jc < nseg) ? 2u : 0u);
-    // Each lane completes the acquire of its own flag before the warp barrier; the barrier
-    // then orders every lane's fetch below after all of them.
-    fence_acquire();
     bool ok = true;
-    if (!__all_sync(0xffffffffu, fearly >= want)) {
-      unsigned fl = 1;
-      if (want != 0 && fearly < want)
-        fl = wait_flag(lane < m ? &lay.rflags[item0 + seg + 1 + lane] : &lay.rflags[item0 + jc],
-                       want, kWaitLimitNs, err);
+    if (fold_early) {
+      cp_async_wait_all();
+    } else {  // wait for the flags not yet set, then fetch (L2 loads: L1 may be stale)
+      const unsigned* flag = lane < m ? &lay.rflags[item0 + seg + 1 + lane] : &lay.rflags[item0 + jc];
+      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, kWaitLimitNs, err) : 1u;
       ok = __all_sync(0xffffffffu, fl != 0);
-    }
-    RevCarry X{0.f, 0.f, 0.f, 0.f};
-    if (jc == nseg && io.ga1 != nullptr && valid) {  // the carry at the end of the sequence
-      const float4 q = lay.ckend[sidx];
-      const float2 e = end_carry(io, sidx, valid, q.z, q.w);
-      X = RevCarry{e.x, e.y, 0.f, 0.f};
-    }
-    if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
-      // Fetch all of it at once (L2 loads: the lines may sit stale in L1), then fold.
-      for (int l = 0; l < 2 * m; ++l)  // map of segment seg + 1 + l / 2, half l % 2
-        sfold[l][lane] = __ldcg(&lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
-      if (jc < nseg) {
-        const float4 q = __ldcg(&lay.carry[(item0 + jc) * 32 + lane]);
-        X = RevCarry{q.x, q.y, q.z, q.w};
+      __syncwarp();  // orders every lane's acquire before every lane's fetch below
+      if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
+        for (int l = 0; l < 2 * m; ++l)
+          sfold[l][lane] = __ldcg(&lay.rmap[((item0 + seg + 1 + (l >> 1)) * 32 + lane) * 2 + (l & 1)]);
+        if (jc < nseg) sfold[2 * m][lane] = __ldcg(&lay.carry[(item0 + jc) * 32 + lane]);
       }
-      __syncwarp();
+    }
+    __syncwarp();
+    RevCarry X{0.f, 0.f, 0.f, 0.f};
+    if (jc == nseg) {  // the carry at the end of the sequence (a later loss's gradient)
+      if (io.ga1 != nullptr && valid) {
+        const float4 q = lay.ckend[sidx];
+        const float2 e = end_carry(io, sidx, valid, q.z, q.w);
+        X = RevCarry{e.x, e.y, 0.f, 0.f};
+      }
+    } else if (ok) {
+      const float4 q = sfold[2 * m][lane];
+      X = RevCarry{q.x, q.y, q.z, q.w};
+    }
+    if (ok)
       for (int l = m - 1; l >= 0; --l)
         X = rev_apply(get_agg(sfold[2 * l][lane], sfold[2 * l + 1][lane]), X);
-    }
     sxe[lane] = make_float4(X.b, X.g, X.bd, X.gd);
   }
   __syncthreads();
