@@ -104,9 +104,9 @@ WKV_API int wkv_forward_bf16(int64_t B, int64_t T, int64_t C, const float* w, co
  * the result of one call over the whole sequence.
  *
  * Long sequences with few channels (B*C small) are split into time segments processed in
- * parallel; the per-segment carries are combined on the device (decoupled look-back with
- * bounded waits). This path allocates its scratch with cudaMallocAsync on `stream` and
- * frees it again in stream order.
+ * parallel; each segment folds the results that earlier segments publish, in a fixed order
+ * (bitwise reproducible), with bounded waits. This path allocates its scratch with
+ * cudaMallocAsync on `stream` and frees it again in stream order.
  */
 WKV_API int wkv_forward_state(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
                               const float* k, const float* v, const float* r, float* y,
@@ -121,7 +121,7 @@ WKV_API int wkv_forward_state(int64_t B, int64_t T, int64_t C, const float* w, c
  * memory, a deployment that forbids dynamic allocation after start-up).
  *
  * Same arguments, layout, semantics and results as wkv_forward_state; the caller passes
- * all inputs and outputs. The scratch of the chunked path (look-back flags and carries,
+ * all inputs and outputs. The scratch of the chunked path (flags and published carries,
  * about 1 KiB per batch row x 32-channel group x 256-token segment) comes from a fixed
  * array of 8 MiB in the library's device memory, which every GPU that loads the library
  * holds until the process exits. Problems whose chunked

@@ -15,8 +15,8 @@ extern "C" {
 
 /*
  * Runs the chunked forward on a small internal problem (B = 1, C = 32, three time
- * segments; every input zero) in which segment 0 withholds its published prefix,
- * so the look-back of the later segments waits on a flag that nothing sets and gives up
+ * segments; every input zero) in which segment 0 withholds its published aggregate, so
+ * the later segments wait for a flag that nothing sets and give up
  * after `wait_ns` nanoseconds (bounded wait; no trap, no hang). The kernel still ends and
  * the next wkv_stream_status(stream) returns WKV_ERR_TIMEOUT, after which the error word
  * is clear again. Allocates its buffers with cudaMallocAsync on `stream` and frees them in

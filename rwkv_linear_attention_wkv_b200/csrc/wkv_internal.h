@@ -51,8 +51,8 @@ int launch_fwd_stream(const FwdArgs& a, bool bf16, bool force_plain, cudaStream_
 size_t chunked_scratch_bytes(int64_t B, int64_t T, int64_t C, int64_t* flag_bytes,
                              int* n_segments);
 int launch_fwd_chunked(const FwdArgs& a, void* scratch, int n_segments, cudaStream_t stream);
-// Same, with the look-back wait limit (ns) given and, for tests of the bounded wait,
-// segment 0 optionally withholding its inclusive prefix so that its successors give up.
+// Same, with the wait limit (ns) given and, for tests of the bounded wait, segment 0
+// optionally withholding its published aggregate so that its successors give up.
 int launch_fwd_chunked_ex(const FwdArgs& a, void* scratch, int n_segments,
                           unsigned long long wait_ns, int withhold_seg0, cudaStream_t stream);
 

@@ -4,7 +4,7 @@
 // they run the operator, e.g. a serving loop that must not risk the implicit device
 // synchronisation an allocation can cause, an application whose memory manager owns all
 // device memory and forbids raw allocations, or a deployment that permits no dynamic
-// allocation once it has started. wkv_forward_state allocates the look-back scratch of its
+// allocation once it has started. wkv_forward_state allocates the scratch of its
 // chunked path with cudaMallocAsync; this variant takes that scratch from a fixed array in
 // the library's own device memory instead.
 //
@@ -87,7 +87,7 @@ extern "C" WKV_API int wkv_forward_state_static(int64_t B, int64_t T, int64_t C,
   int rc = WKV_OK;
   void* scratch = static_scratch(&rc);
   if (scratch == nullptr) return rc;
-  // The look-back flags and the segment ticket must start at zero; the rest of the
+  // The flags and the segment ticket must start at zero; the rest of the
   // scratch is written before it is read.
   if (cudaMemsetAsync(scratch, 0, size_t(flag_bytes), stream) != cudaSuccess) return WKV_ERR_CUDA;
   return launch_fwd_chunked(a, scratch, nseg, stream);

@@ -11,16 +11,19 @@
 // (hi, lo) so that a long chain of combinations does not drift.
 //
 // One CTA = W warps x 32 channels of one batch row, covering one segment of W x LS tokens;
-// warp w owns sub-chunk w (LS tokens). Single pass, 16 bytes of HBM traffic per element:
+// warp w owns sub-chunk w (LS tokens). CTAs take segments in ticket order, so every segment
+// a CTA waits for belongs to a CTA that started earlier. Single pass, 16 bytes of HBM
+// traffic per element:
 //   1. every warp TMA-loads its k, v, r sub-tile into shared memory (kept resident) and
 //      folds k, v into the sub-chunk aggregate from the empty state;
-//   2. warp 0 combines the W aggregates, publishes the segment aggregate, walks back over
-//      the predecessors' published aggregates / inclusive prefixes (decoupled look-back;
-//      CTAs take segments in ticket order, so every predecessor is already resident or
-//      done) and publishes the inclusive prefix; each warp then forms its own carry-in;
-//   3. every warp re-runs its sub-chunk from the carry-in out of shared memory, writes y
-//      in place of k and TMA-stores it. The warp holding the last token writes the final
-//      state.
+//   2. warp 0 combines the W aggregates and publishes the segment's aggregate; the last
+//      warp forms the state entering the segment in a fixed order from the published
+//      aggregates of up to kFold earlier segments and the state entering the first of
+//      them (so the result is bitwise reproducible, unlike a look-back that takes whichever
+//      earlier result happens to be ready);
+//   3. every warp combines that state with the aggregates of the sub-chunks before its own,
+//      re-runs its sub-chunk from there out of shared memory, writes y in place of k and
+//      TMA-stores it. The warp holding the last token writes the final state.
 // Every wait is bounded in wall time; a wait that gives up flags the error word and
 // carries on with an empty carry (the result is then wrong, but the kernel ends).
 #include "wkv_internal.h"
@@ -48,14 +51,15 @@ namespace {
 #endif
 constexpr int kW = WKV_SCAN_W;     // warps per CTA (sub-chunks per segment)
 constexpr int kLS = WKV_SCAN_LS;   // tokens per sub-chunk
+constexpr int kFold = 16;          // earlier segments folded in directly (see the kernel)
 constexpr int kSeg = kW * kLS;
 constexpr int64_t kChunkBelowChannels = WKV_SCAN_MIN_CH;
 
 struct ScanLayout {
   unsigned* ticket;
-  unsigned* flags;  // [nbg * nseg]: 0 none, 1 aggregate, 2 inclusive prefix
-  float4* agg;      // [nbg * nseg * 32]
-  float4* incl;     // [nbg * nseg * 32]
+  unsigned* flags;  // [nbg * nseg]: 0 none, 1 aggregate, 2 entering state published
+  float4* agg;      // [nbg * nseg * 32]: the segment's aggregate from the empty state
+  float4* incl;     // [nbg * nseg * 32]: the state entering the segment (fold starts only)
 };
 
 __host__ __device__ inline int64_t scan_flag_bytes(int64_t nitems) {
@@ -87,8 +91,9 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   float* sv = sk + kW * kTile;
   float* sr = sv + kW * kTile;
   float4* sagg = reinterpret_cast<float4*>(sr + (GATE ? kW * kTile : 0));  // [W][32]
-  float4* scarry = sagg + kW * 32;                                         // [32]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(scarry + 32);                // [W]
+  float4* sin = sagg + kW * 32;                                            // [32]
+  float4* sfold = sin + 32;                                                // [kFold][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sfold + kFold * 32);         // [W]
   __shared__ unsigned s_ticket;
 
   const int G = (C + 31) >> 5;
@@ -105,6 +110,9 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   const int g = int(bg - int64_t(b) * G);
   const int c = (g << 5) + lane;
   const bool valid = c < C;
+  const int64_t item0 = bg * nseg;
+  const int64_t item = item0 + seg;
+  const size_t sidx = size_t(b) * C + c;
 
   const int t0 = seg * kSeg + warp * kLS;           // first token of this warp
   const int n = max(0, min(kLS, T - t0));           // tokens of this warp
@@ -126,10 +134,34 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   const float* V = sv + warp * kTile + lane;
   const float* R = sr + warp * kTile + lane;
   float* Y = sk + warp * kTile + lane;
+  const int rb = window_tokens(cp.w2, 128.f);
+
+  // The state entering the segment is formed in a fixed order (bitwise reproducible):
+  // the state entering segment j0 = max(0, seg - kFold) (published by that segment; the
+  // initial state for j0 = 0), then the published aggregates of segments j0 .. seg-1. Only
+  // j0 > 0 waits for another segment's fold, so one link of a serial chain spans kFold
+  // segments. The last warp checks the flags now (one acquire load per lane, while the
+  // tiles load) and, if all are set, copies the inputs into shared memory (cp.async)
+  // while the aggregates are formed; otherwise it waits for them after that.
+  const int j0 = max(0, seg - kFold);
+  const int mfold = seg - j0;  // aggregates to fold
+  const unsigned fwant = lane < mfold ? 1u : ((lane == 31 && j0 > 0) ? 2u : 0u);
+  const unsigned* fflag = lane < mfold ? &lay.flags[item0 + j0 + lane] : &lay.flags[item0 + j0];
+  bool fold_early = false;
+  if (warp == kW - 1) {
+    const unsigned fl = fwant != 0 ? ld_acquire(fflag) : 0u;
+    fold_early = __all_sync(0xffffffffu, fl >= fwant);
+    __syncwarp();  // orders every lane's acquire before every lane's copies below
+    if (fold_early) {
+      for (int l = 0; l < mfold; ++l) cp_async_16(&sfold[l * 32 + lane], &lay.agg[(item0 + j0 + l) * 32 + lane]);
+      if (j0 > 0) cp_async_16(&sin[lane], &lay.incl[(item0 + j0) * 32 + lane]);
+      cp_async_commit();
+    }
+  }
 
   // ---- 1. sub-chunk aggregate from the empty state ----
-  const int rb = window_tokens(cp.w2, 128.f);
   if (n > 0) mbar_wait(bar, 0, err);
+  __syncwarp();
   ChanState s = empty_state();
   {
     int j = 0;
@@ -146,75 +178,62 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   sagg[warp * 32 + lane] = make_float4(mine.a, mine.b, mine.ph, mine.pl);
   __syncthreads();
 
-  // ---- 2. segment aggregate, look-back, carries ----
-  if (warp == 0) {
-    auto ld = [&](const float4& q) { return Agg{q.x, q.y, q.z, q.w}; };
-    Agg A = ld(sagg[lane]);
-    for (int i = 1; i < kW; ++i) {
-      const int ni = max(0, min(kLS, T - (seg * kSeg + i * kLS)));
-      A = combine(A, ld(sagg[i * 32 + lane]), float(ni), cp.w2);
+  // ---- 2. the segment's aggregate; the state entering the segment ----
+  if (warp == 0 && seg + 1 < nseg && !(withhold_seg0 && seg == 0)) {
+    Agg A = agg_empty();
+    for (int i = 0; i < kW; ++i) {
+      const float4 q = sagg[i * 32 + lane];
+      A = combine(A, Agg{q.x, q.y, q.z, q.w}, float(kLS), cp.w2);  // all sub-chunks full
     }
-    const int seg_len = min(kSeg, T - seg * kSeg);
-    const int64_t item = bg * nseg + seg;
-    Agg carry;
-    if (seg == 0) {
-      const size_t sidx = size_t(b) * C + c;
-      carry = (a0 != nullptr && valid) ? to_agg(load_state(a0[sidx], b0[sidx], p0[sidx]))
-                                       : agg_empty();
-    } else {
-      lay.agg[item * 32 + lane] = make_float4(A.a, A.b, A.ph, A.pl);
-      warp_publish(&lay.flags[item], 1u);
-      // Walk back: acc covers the segments between j and seg (exclusive), all full.
-      Agg acc = agg_empty();
-      int covered = 0;
-      carry = agg_empty();
-      for (int j = seg - 1; j >= 0; --j) {
-        const int64_t pj = bg * nseg + j;
-        unsigned f = 0;
-        if (lane == 0) {
-          f = ld_acquire(&lay.flags[pj]);
-          if (f == 0) {
-            const uint64_t start = global_ns();
-            while ((f = ld_acquire(&lay.flags[pj])) == 0) {
-              if (global_ns() - start > wait_ns) break;
-              __nanosleep(64);
-            }
-            if (f == 0) atomicOr(err, kErrTimeout);
-          }
-        }
-        f = __shfl_sync(0xffffffffu, f, 0);
-        __syncwarp();
-        if (f == 0) {  // gave up: continue from an empty carry
-          carry = acc;
-          break;
-        }
-        // L2 loads (.cg): the line may sit stale in this SM's L1 from an earlier read.
-        const float4 q = (f == 2) ? __ldcg(&lay.incl[pj * 32 + lane]) : __ldcg(&lay.agg[pj * 32 + lane]);
-        acc = combine(ld(q), acc, float(covered), cp.w2);
-        covered += kSeg;
-        if (f == 2) {
-          carry = acc;
-          break;
-        }
-        if (j == 0) carry = acc;  // unreachable: segment 0 publishes only inclusive
+    lay.agg[item * 32 + lane] = make_float4(A.a, A.b, A.ph, A.pl);
+    warp_publish(&lay.flags[item], 1u);
+  }
+  if (warp == kW - 1) {
+    bool ok = true;
+    if (fold_early) {
+      cp_async_wait_all();
+    } else {  // wait for the flags not yet set, then fetch (L2 loads: L1 may be stale)
+      const unsigned fl = fwant != 0 ? wait_flag(fflag, fwant, wait_ns, err) : 1u;
+      ok = __all_sync(0xffffffffu, fl != 0);
+      __syncwarp();  // orders every lane's acquire before every lane's fetch below
+      if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
+        for (int l = 0; l < mfold; ++l) sfold[l * 32 + lane] = __ldcg(&lay.agg[(item0 + j0 + l) * 32 + lane]);
+        if (j0 > 0) sin[lane] = __ldcg(&lay.incl[(item0 + j0) * 32 + lane]);
       }
     }
-    const Agg incl = combine(carry, A, float(seg_len), cp.w2);
-    if (!(withhold_seg0 && seg == 0)) {
-      lay.incl[item * 32 + lane] = make_float4(incl.a, incl.b, incl.ph, incl.pl);
-      warp_publish(&lay.flags[item], 2u);
+    __syncwarp();
+    Agg X = agg_empty();
+    if (j0 == 0) {
+      if (a0 != nullptr && valid) X = to_agg(load_state(a0[sidx], b0[sidx], p0[sidx]));
+    } else if (ok) {
+      const float4 q = sin[lane];
+      X = Agg{q.x, q.y, q.z, q.w};
     }
-    scarry[lane] = make_float4(carry.a, carry.b, carry.ph, carry.pl);
+    if (ok)
+      for (int l = 0; l < mfold; ++l) {
+        const float4 a = sfold[l * 32 + lane];
+        X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kSeg), cp.w2);
+      }
+    __syncwarp();
+    sin[lane] = make_float4(X.a, X.b, X.ph, X.pl);
   }
   __syncthreads();
 
-  // ---- 3. re-run the sub-chunk from its carry-in, write y ----
+  // ---- 3. each warp's carry-in; re-run the sub-chunk from it, write y ----
+  Agg cin;
   {
-    auto ld = [&](const float4& q) { return Agg{q.x, q.y, q.z, q.w}; };
-    Agg cin = ld(scarry[lane]);
-    for (int i = 0; i < warp; ++i) cin = combine(cin, ld(sagg[i * 32 + lane]), float(kLS), cp.w2);
-    s = to_state(cin);
+    const float4 q = sin[lane];
+    cin = Agg{q.x, q.y, q.z, q.w};
   }
+  if (warp == 0 && seg > 0 && seg + kFold < nseg) {  // segment seg + kFold starts here
+    lay.incl[item * 32 + lane] = make_float4(cin.a, cin.b, cin.ph, cin.pl);
+    warp_publish(&lay.flags[item], 2u);
+  }
+  for (int i = 0; i < warp; ++i) {
+    const float4 q = sagg[i * 32 + lane];
+    cin = combine(cin, Agg{q.x, q.y, q.z, q.w}, float(kLS), cp.w2);
+  }
+  s = to_state(cin);
   if (n > 0) {
     const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
     int j = 0;
@@ -233,10 +252,10 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
     if (lane == 0) {
       tma_store_3d(&tm_y, sk + warp * kTile, g << 5, t0, b);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read<0>();  // the tile stays until the store has read it
     }
+    __syncwarp();
     if (a1 != nullptr && valid && t0 + n == T) {
-      const size_t sidx = size_t(b) * C + c;
       a1[sidx] = s.a;
       b1[sidx] = s.b;
       p1[sidx] = state_log_scale(s);
@@ -262,8 +281,8 @@ size_t chunked_scratch_bytes(int64_t B, int64_t T, int64_t C, int64_t* flag_byte
 }
 
 static size_t chunked_smem_bytes(bool gate) {
-  return size_t(gate ? 3 : 2) * kW * kLS * 32 * sizeof(float) + (kW * 32 + 32) * sizeof(float4) +
-         kW * sizeof(uint64_t);
+  return size_t(gate ? 3 : 2) * kW * kLS * 32 * sizeof(float) +
+         (kW * 32 + 32 + kFold * 32) * sizeof(float4) + kW * sizeof(uint64_t);
 }
 
 int launch_fwd_chunked_ex(const FwdArgs& a, void* scratch, int nseg, unsigned long long wait_ns,

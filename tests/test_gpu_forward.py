@@ -191,6 +191,10 @@ def test_long_context_full_size_with_state(W):
     ref, A, Bd = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r, want_state=True)
     assert_fp32_close(y.cpu().numpy(), ref)
     assert_state_close(a1.cpu().numpy(), b1.cpu().numpy(), p1.cpu().numpy(), A, Bd)
+    # The segments' carries are folded in a fixed order: a second call gives the same bits.
+    y2, (a2, b2, p2) = W.wkv_forward_state(w, u, k, v, r)
+    for one, two in ((y, y2), (a1, a2), (b1, b2), (p1, p2)):
+        assert torch.equal(one, two)
 
 
 def test_long_context_stress_distributions(W):

@@ -3,7 +3,7 @@
 Some callers cannot allocate device memory at the point where they run the operator: a
 serving loop that must not risk the implicit device synchronisation an allocation can
 bring, an application whose memory manager owns all device memory, or a deployment that
-forbids dynamic allocation once started. For them the library keeps the look-back scratch
+forbids dynamic allocation once started. For them the library keeps the chunked path's scratch
 of the chunked path in a fixed 8 MiB array of its own device memory instead of allocating
 it per call. This test calls that entry point through the C ABI and checks it against
 wkv_forward_state on two calls in a row (the second reuses the scratch the first left
@@ -70,7 +70,7 @@ def test_static_scratch_matches_allocating_entry_point_twice(W):
 
 
 def test_static_scratch_rejects_problems_beyond_its_size(W):
-    # One sequence of 65536 tokens x 4096 channels needs about 33 MiB of look-back scratch.
+    # One sequence of 65536 tokens x 4096 channels needs about 33 MiB of scratch.
     B, T, C = 1, 65536, 4096
     fake = ctypes.c_void_p(1 << 20)   # never dereferenced: the size check comes first
     rc = W.lib.wkv_forward_state_static(B, T, C, *([fake] * 6), None, None, None,
