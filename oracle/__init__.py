@@ -8,8 +8,9 @@ Two parts:
 
 * ``wkv_oracle.c`` (built into ``libwkv_oracle.so`` by :func:`build`), plain C in
   double precision: the O(T^2) parallel form, the unstabilised recurrence, the decode
-  step, the analytic backward and the backward through an entering and leaving state
-  (the recurrence's adjoint);
+  step, the analytic backward, the backward through an entering and leaving state (the
+  recurrence's adjoint), and RWKV-7's generalised-delta-rule recurrence (research report
+  "RWKV模型深度研究报告", section 1.3.3);
 * a few NumPy routines for tiny inputs that restate the operator through other
   routes: a causal softmax over logits (the operator as attention with
   query-independent weights), and one inference step written from the single-token
@@ -55,8 +56,10 @@ def _load():
         lib.oracle_wkv_decode.argtypes = [I, I, I] + [P] * 8
         lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 13
         lib.oracle_wkv_backward_state.argtypes = [I, I, I] + [P] * 21
+        lib.oracle_wkv7_recurrent.argtypes = [I, I, I, I] + [P] * 9
         for f in (lib.oracle_wkv_direct, lib.oracle_wkv_recurrent, lib.oracle_wkv_decode,
-                  lib.oracle_wkv_backward, lib.oracle_wkv_backward_state):
+                  lib.oracle_wkv_backward, lib.oracle_wkv_backward_state,
+                  lib.oracle_wkv7_recurrent):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -147,6 +150,18 @@ def wkv_backward_state(w, u, k, v, r, dy, A0=None, B0=None, gA=None, gB=None):
         _ptr(dB0), _ptr(dwa), _ptr(dua), _ptr(dA0a), _ptr(dB0a)))
     return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dA0": dA0, "dB0": dB0,
             "dw_abs": dwa, "du_abs": dua, "dA0_abs": dA0a, "dB0_abs": dB0a}
+
+
+def wkv7_recurrent(r, w, k, v, a, b, S0=None, want_state=False):
+    """RWKV-7 generalised-delta-rule recurrence per head; r, w, k, v, a, b (B, T, H, N),
+    S0 (B, H, N, N) or None. Returns y (B, T, H, N), or (y, S_T) with want_state."""
+    r, w, k, v, a, b, S0 = map(_f64, (r, w, k, v, a, b, S0))
+    B, T, H, N = k.shape
+    y = np.empty((B, T, H, N))
+    S1 = np.empty((B, H, N, N)) if want_state else None
+    _check(_load().oracle_wkv7_recurrent(B, T, H, N, _ptr(r), _ptr(w), _ptr(k), _ptr(v),
+                                         _ptr(a), _ptr(b), _ptr(y), _ptr(S0), _ptr(S1)))
+    return (y, S1) if want_state else y
 
 
 def state_from_scaled(a, b, p):

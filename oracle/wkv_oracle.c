@@ -316,3 +316,53 @@ int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
     free(Aprev); free(Bprev); free(Aabs); free(D); free(wkv);
     return 0;
 }
+
+/*
+ * O6: RWKV-7's generalised-delta-rule state update, per head, as written in the research
+ * report "RWKV模型深度研究报告（截至2026年初）", section 1.3.3 "RWKV-7 (Goose)":
+ *   S_t = S_{t-1} (diag(w_t) + a_t^T b_t) + v_t^T k_t
+ * with row vectors w_t (the decay, per key channel), a_t, b_t, k_t, v_t of the head size N,
+ * so S is N x N (row i: value channel, column j: key channel):
+ *   S_t[i][j] = S_{t-1}[i][j] w_t[j] + (sum_l S_{t-1}[i][l] a_t[l]) b_t[j] + v_t[i] k_t[j].
+ * The report gives no read-out; the reading used is the linear-attention one with the
+ * receptance as the query: y_t = S_t r_t^T, y_t[i] = sum_j S_t[i][j] r_t[j].
+ * Layout: r, w, k, v, a, b, y are (B, T, H, N) row-major; the state S0 (may be NULL =
+ * zero) and S1 (may be NULL = not wanted) are (B, H, N, N) with S[i][j] at i * N + j.
+ */
+int oracle_wkv7_recurrent(int64_t B, int64_t T, int64_t H, int64_t N, const double *r,
+                          const double *w, const double *k, const double *v, const double *a,
+                          const double *b, double *y, const double *S0, double *S1)
+{
+    if (B < 0 || T < 0 || H < 0 || N < 0) return -1;
+    if (T > 0 && (!r || !w || !k || !v || !a || !b || !y)) return -1;
+    double *S = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N * N : 1));
+    double *sa = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+    if (!S || !sa) { free(S); free(sa); return -1; }
+    for (int64_t bb = 0; bb < B; ++bb)
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t s_off = (bb * H + h) * N * N;
+            for (int64_t e = 0; e < N * N; ++e) S[e] = S0 ? S0[s_off + e] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t off = ((bb * T + t) * H + h) * N;
+                for (int64_t i = 0; i < N; ++i) {            /* S_{t-1} a_t^T */
+                    double acc = 0.0;
+                    for (int64_t l = 0; l < N; ++l) acc += S[i * N + l] * a[off + l];
+                    sa[i] = acc;
+                }
+                for (int64_t i = 0; i < N; ++i)
+                    for (int64_t j = 0; j < N; ++j)
+                        S[i * N + j] = S[i * N + j] * w[off + j] + sa[i] * b[off + j]
+                                     + v[off + i] * k[off + j];
+                for (int64_t i = 0; i < N; ++i) {            /* y_t = S_t r_t^T */
+                    double acc = 0.0;
+                    for (int64_t j = 0; j < N; ++j) acc += S[i * N + j] * r[off + j];
+                    y[off + i] = acc;
+                }
+            }
+            if (S1)
+                for (int64_t e = 0; e < N * N; ++e) S1[s_off + e] = S[e];
+        }
+    free(S);
+    free(sa);
+    return 0;
+}

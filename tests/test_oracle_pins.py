@@ -334,3 +334,94 @@ def test_backward_state_chains_over_a_split_sequence():
         np.testing.assert_allclose(first[n] + second[n], whole[n], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(first["dA0"], whole["dA0"], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(first["dB0"], whole["dB0"], rtol=1e-11, atol=1e-12)
+
+
+# ---- RWKV-7 generalised-delta-rule recurrence (research report, section 1.3.3) ----
+
+def _unit_rows(g, shape):
+    x = g.standard_normal(shape)
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def test_wkv7_delta_rule_stores_the_latest_pair():
+    # w = 1, a = -k^, b = k^ (unit k^) makes the transition I - k^T k^, so after each token
+    # the state maps the token's key exactly to its value: S_t k^_t^T = v_t. Reading the
+    # state with r_t = k^_t therefore returns v_t, whatever came before.
+    g = np.random.Generator(np.random.PCG64(40))
+    B, T, H, N = 2, 9, 3, 6
+    kh = _unit_rows(g, (B, T, H, N))
+    v = g.standard_normal((B, T, H, N))
+    S0 = g.standard_normal((B, H, N, N))
+    y = oracle.wkv7_recurrent(kh, np.ones((B, T, H, N)), kh, v, -kh, kh, S0)
+    np.testing.assert_allclose(y, v, rtol=1e-12, atol=1e-12)
+
+
+def test_wkv7_reflection_preserves_the_state_norm():
+    # w = 1, a = -2 k^, b = k^: the transition I - 2 k^T k^ is a reflection (orthogonal), so
+    # with v = 0 every row of S keeps its length; with k = 0 nothing is written.
+    g = np.random.Generator(np.random.PCG64(41))
+    B, T, H, N = 1, 12, 2, 5
+    kh = _unit_rows(g, (B, T, H, N))
+    S0 = g.standard_normal((B, H, N, N))
+    zero = np.zeros((B, T, H, N))
+    _, ST = oracle.wkv7_recurrent(zero, np.ones((B, T, H, N)), zero, zero, -2 * kh, kh, S0,
+                                  want_state=True)
+    np.testing.assert_allclose(np.linalg.norm(ST, axis=-1), np.linalg.norm(S0, axis=-1),
+                               rtol=1e-12)
+
+
+def test_wkv7_without_delta_term_is_decayed_linear_attention():
+    # a = b = 0: S_t = sum_{s<=t} v_s^T (k_s * D_{s,t}) with D_{s,t} = prod_{s<u<=t} w_u (per key
+    # channel), so y_t = sum_{s<=t} v_s <k_s * D_{s,t}, r_t>: attention with per-channel
+    # decayed scores, summed here pair by pair.
+    g = np.random.Generator(np.random.PCG64(42))
+    B, T, H, N = 2, 7, 2, 4
+    r, k, v = (g.standard_normal((B, T, H, N)) for _ in range(3))
+    w = g.uniform(0.3, 1.0, (B, T, H, N))
+    zero = np.zeros((B, T, H, N))
+    y = oracle.wkv7_recurrent(r, w, k, v, zero, zero)
+    ref = np.zeros_like(y)
+    for bb in range(B):
+        for h in range(H):
+            for t in range(T):
+                for s in range(t + 1):
+                    D = np.prod(w[bb, s + 1:t + 1, h], axis=0) if t > s else np.ones(N)
+                    ref[bb, t, h] += v[bb, s, h] * np.dot(k[bb, s, h] * D, r[bb, t, h])
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_wkv7_scalar_head_closed_form():
+    # N = 1: s_t = s_{t-1} (w_t + a_t b_t) + v_t k_t, a scalar linear recurrence with the
+    # closed form s_T = s_0 prod_t m_t + sum_i v_i k_i prod_{j>i} m_j, m = w + a b.
+    g = np.random.Generator(np.random.PCG64(43))
+    T = 15
+    r, k, v, a, b = (g.standard_normal((1, T, 1, 1)) for _ in range(5))
+    w = g.uniform(0.2, 1.0, (1, T, 1, 1))
+    s0 = np.array([[[[0.7]]]])
+    y, sT = oracle.wkv7_recurrent(r, w, k, v, a, b, s0, want_state=True)
+    m = (w + a * b)[0, :, 0, 0]
+    vk = (v * k)[0, :, 0, 0]
+    for t in range(T):
+        st = s0[0, 0, 0, 0] * np.prod(m[:t + 1]) + sum(vk[i] * np.prod(m[i + 1:t + 1])
+                                                       for i in range(t + 1))
+        assert y[0, t, 0, 0] == pytest.approx(st * r[0, t, 0, 0], rel=1e-12, abs=1e-14)
+    assert sT[0, 0, 0, 0] == pytest.approx(s0[0, 0, 0, 0] * np.prod(m)
+                                           + sum(vk[i] * np.prod(m[i + 1:]) for i in range(T)),
+                                           rel=1e-12)
+
+
+def test_wkv7_split_with_state_handover():
+    g = np.random.Generator(np.random.PCG64(44))
+    B, T, H, N, T1 = 2, 20, 2, 5, 8
+    r, k, v = (g.standard_normal((B, T, H, N)) for _ in range(3))
+    w = g.uniform(0.5, 1.0, (B, T, H, N))
+    kh = _unit_rows(g, (B, T, H, N))
+    a, b = -kh, kh * g.uniform(0, 1, (B, T, H, 1))
+    S0 = g.standard_normal((B, H, N, N))
+    y, ST = oracle.wkv7_recurrent(r, w, k, v, a, b, S0, want_state=True)
+    y1, S1 = oracle.wkv7_recurrent(r[:, :T1], w[:, :T1], k[:, :T1], v[:, :T1], a[:, :T1],
+                                   b[:, :T1], S0, want_state=True)
+    y2, S2 = oracle.wkv7_recurrent(r[:, T1:], w[:, T1:], k[:, T1:], v[:, T1:], a[:, T1:],
+                                   b[:, T1:], S1, want_state=True)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(S2, ST, rtol=1e-13, atol=1e-13)
