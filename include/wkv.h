@@ -205,6 +205,24 @@ WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, 
                                cudaStream_t stream);
 
 /*
+ * RWKV-7 recurrence per head, fp32 (research report "RWKV模型深度研究报告（截至2026年初）",
+ * section 1.3.3 "RWKV-7 (Goose)": the generalised-delta-rule state update
+ *   S_t = S_{t-1} (diag(w_t) + a_t^T b_t) + v_t^T k_t
+ * with an N x N state per head, row i = value channel, column j = key channel). The
+ * report gives no read-out; the output is y_t = S_t r_t^T (the receptance as the query).
+ *   r, w, k, v, a, b, y: fp32 (B, T, H, N) row-major (C = H N channels, head h holding
+ *     channels h N .. h N + N - 1); w is the decay factor itself (typically in (0, 1)).
+ *   s0: the initial state, fp32 (B, H, N, N) with S[i][j] at i N + j; NULL = zero.
+ *   s1: the final state, same layout; NULL = not wanted; may alias s0.
+ * N must be 64 (else WKV_ERR_UNSUPPORTED); every pointer must be 16-byte aligned (else
+ * WKV_ERR_ALIGNMENT). T == 0: s1 = s0 (zero if s0 is NULL). Asynchronous on `stream`.
+ */
+WKV_API int wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float* r,
+                         const float* w, const float* k, const float* v, const float* a,
+                         const float* b, float* y, const float* s0, float* s1,
+                         cudaStream_t stream);
+
+/*
  * Query and clear device-side errors. Synchronises `stream`, then returns WKV_ERR_TIMEOUT
  * if any kernel of this library on the current device gave up a bounded wait since the
  * last query (the outputs of that call are then undefined), WKV_ERR_CUDA if the stream

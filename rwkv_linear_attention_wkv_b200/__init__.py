@@ -13,7 +13,8 @@ import os
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
            "wkv_backward", "wkv_backward_state", "wkv_backward_workspace_bytes",
-           "wkv_stream_status", "wkv_status_string", "WkvError", "lib", "LIB_PATH"]
+           "wkv7_forward", "wkv_stream_status", "wkv_status_string", "WkvError", "lib",
+           "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
 
@@ -39,6 +40,7 @@ _SIGS = {
     "wkv_testing_backward_plain": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P],
                                    ctypes.c_int),
     "wkv_backward_state": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "wkv7_forward": ([_I, _I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
     "wkv_testing_backward_state_plain": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
                                          ctypes.c_int),
     "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
@@ -278,6 +280,33 @@ def wkv_backward_state(w, u, k, v, r, dy, state=None, grad_state=None, want_dr=T
           _ptr(out["da0"]), _ptr(out["db0"]), _ptr(out["dp0"]),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return out
+
+
+def wkv7_forward(r, w, k, v, a, b, state=None, y=None, state_out=None, want_state=True,
+                 stream=None):
+    """RWKV-7 recurrence per head: r, w, k, v, a, b fp32 (B, T, H, N), N = 64; state
+    (B, H, N, N) or None (zero). Returns (y, S_T), or (y, None) with want_state=False.
+    state_out may be given (and may be `state` itself)."""
+    torch = _torch()
+    f32 = torch.float32
+    if k.dim() != 4:
+        raise ValueError("k must be (B, T, H, N)")
+    B, T, H, N = k.shape
+    for n, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b)):
+        _need(t, n, f32, (B, T, H, N))
+    if y is None:
+        y = torch.empty((B, T, H, N), dtype=f32, device=k.device)
+    _need(y, "y", f32, (B, T, H, N))
+    if state is not None:
+        _need(state, "state", f32, (B, H, N, N))
+    s1 = None
+    if want_state:
+        s1 = state_out if state_out is not None else torch.empty((B, H, N, N), dtype=f32,
+                                                                 device=k.device)
+        _need(s1, "state_out", f32, (B, H, N, N))
+    _call("wkv7_forward", B, T, H, N, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+          _ptr(y), _ptr(state), _ptr(s1), _stream(stream))
+    return y, s1
 
 
 def wkv_stream_status(stream=None) -> int:

@@ -270,6 +270,32 @@ WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, 
                        workspace_bytes, false, stream, st);
 }
 
+WKV_API int wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float* r,
+                         const float* w, const float* k, const float* v, const float* a,
+                         const float* b, float* y, const float* s0, float* s1,
+                         cudaStream_t stream) {
+  if (B < 0 || T < 0 || H < 0 || N < 0) return WKV_ERR_INVALID_ARG;
+  if (B == 0 || H == 0) return WKV_OK;
+  if (N != 64) return WKV_ERR_UNSUPPORTED;
+  if (T > 0 && (!r || !w || !k || !v || !a || !b || !y)) return WKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {r, w, k, v, a, b, y, s0, s1};
+  for (const void* q : ptrs)
+    if (!aligned(q, 16)) return WKV_ERR_ALIGNMENT;
+  if (T >= (int64_t(1) << 31) || B * H >= (int64_t(1) << 31) || H >= (int64_t(1) << 24) ||
+      B > INT64_MAX / T / (H * N))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t sbytes = size_t(B) * H * N * N * sizeof(float);
+  if (T == 0) {  // no tokens: the state passes through
+    if (s1 == nullptr || s1 == s0) return WKV_OK;
+    const cudaError_t e = s0 ? cudaMemcpyAsync(s1, s0, sbytes, cudaMemcpyDeviceToDevice, stream)
+                             : cudaMemsetAsync(s1, 0, sbytes, stream);
+    return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  }
+  unsigned* err = error_word();
+  if (err == nullptr) return WKV_ERR_CUDA;
+  return launch_wkv7(B, T, H, r, w, k, v, a, b, y, s0, s1, err, stream);
+}
+
 WKV_API int wkv_stream_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV_ERR_CUDA;
   unsigned* err = error_word();

@@ -106,4 +106,9 @@ int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);
 // T == 0 with the state's gradients wanted: they pass straight through.
 int launch_backward_no_tokens(const BwdArgs& a, cudaStream_t stream);
 
+// RWKV-7 recurrence (wkv7.cu), head size 64, all pointers 16-byte aligned.
+int launch_wkv7(int64_t B, int64_t T, int64_t H, const float* r, const float* w, const float* k,
+                const float* v, const float* a, const float* b, float* y, const float* s0,
+                float* s1, unsigned* err, cudaStream_t stream);
+
 }  // namespace wkv

@@ -170,3 +170,44 @@ def sample_channels(B: int, C: int, n: int, seed: int = 12345):
     n = min(n, B * C)
     flat = g.choice(B * C, size=n, replace=False)
     return [(int(f // C), int(f % C)) for f in np.sort(flat)]
+
+
+@dataclass
+class Wkv7Inputs:
+    """One seeded RWKV-7 problem: (B, T, H, N) float32 tensors and an initial state."""
+
+    B: int
+    T: int
+    H: int
+    N: int
+    r: np.ndarray
+    w: np.ndarray      # decay factor in (0.5, 1]
+    k: np.ndarray
+    v: np.ndarray
+    a: np.ndarray      # -kappa^ (unit per head and token)
+    b: np.ndarray      # kappa^ * alpha, alpha ~ U(0, 1) per channel
+    S0: np.ndarray     # (B, H, N, N)
+
+
+def rwkv7_inputs(B: int, T: int, H: int, N: int = 64, seed: int = 0) -> Wkv7Inputs:
+    """RWKV-7 recurrence inputs (research report, section 1.3.3: decay w_t, in-context
+    learning vectors a_t, b_t). Draw order from PCG64(seed): r, k, v ~ N(0, 1); w = exp(-x)
+    with x ~ U(0, 0.7); kappa ~ N(0, 1) normalised per (b, t, h) to kappa^; alpha ~ U(0, 1);
+    a = -kappa^, b = kappa^ alpha (the delta rule's removal of the old value along kappa^,
+    so the transition diag(w) + a^T b stays contracting); S0 ~ N(0, 0.1). All float32."""
+    g = np.random.Generator(np.random.PCG64(seed))
+    shape = (B, T, H, N)
+
+    def normal(scale=1.0):
+        x = g.standard_normal(shape, dtype=np.float32)
+        return x if scale == 1.0 else x * np.float32(scale)
+
+    r, k, v = normal(), normal(), normal()
+    w = np.exp(-g.uniform(0.0, 0.7, size=shape)).astype(np.float32)
+    kap = normal()
+    kap /= np.linalg.norm(kap, axis=-1, keepdims=True)
+    alpha = g.uniform(0.0, 1.0, size=shape).astype(np.float32)
+    a = -kap
+    b = (kap * alpha).astype(np.float32)
+    S0 = g.standard_normal((B, H, N, N), dtype=np.float32) * np.float32(0.1)
+    return Wkv7Inputs(B, T, H, N, r, w, k, v, a.astype(np.float32), b, S0)
