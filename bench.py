@@ -444,6 +444,25 @@ def run_workload(args):
                         args.warmup, stream)
         line("decode", "decode step fp32 256 seq x 32 layers x 4096 (state in place)", ms, n,
              40 * n, {"tokens_per_s": dd.N / (ms / 1e3)})
+    elif args.workload == "rwkv7":
+        T7 = args.seq or 4096
+        x = wkv_inputs.rwkv7_inputs(8, T7, 64, seed=0)
+        t = {nm: d(getattr(x, nm)) for nm in ("r", "w", "k", "v", "a", "b")}
+        s0 = d(x.S0)
+        y = torch.empty_like(t["k"])
+        s1 = torch.empty_like(s0)
+        n = x.B * x.T * x.H * x.N
+        ms = _time_loop(lambda: W.wkv7_forward(*(t[nm] for nm in "rwkvab"), state=s0, y=y,
+                                               state_out=s1), args.steps, args.warmup, stream)
+        # FP32 work per token and head: sa (N^2 FMA), update (N^2 FMUL + 2 N^2 FMA), y (N^2 FMA)
+        flops = 9 * x.N * x.N * x.B * x.T * x.H
+        # FP32 peak from unit counts: 148 SMs x 128 FMA lanes x 2 x the max SM clock
+        alu_peak = 148 * 128 * 2 * 1.965e9
+        line("rwkv7", f"RWKV-7 recurrence fp32 8x{x.T}x64 heads x 64 (state in and out)", ms, n,
+             28 * n + 8 * x.B * x.H * x.N * x.N,
+             {"flops": flops, "achieved_TFLOPs": flops / (ms / 1e3) / 1e12,
+              "alu_peak_TFLOPs": alu_peak / 1e12,
+              "alu_frac": flops / (ms / 1e3) / alu_peak})
     else:
         raise SystemExit(f"unknown workload {args.workload}")
     if W.wkv_stream_status() != 0:
@@ -461,7 +480,7 @@ def main():
                     help="batch rows per GPU (default 8, the measured workload; smaller "
                          "values are for profiler captures)")
     ap.add_argument("--workload", default="bf16_7b",
-                    choices=["bf16_7b", "train_169m", "long_ctx", "decode"],
+                    choices=["bf16_7b", "train_169m", "long_ctx", "decode", "rwkv7"],
                     help="bf16_7b (default) prints the benchmark line; the others print "
                          "measurements of the other workloads, one GPU")
     ap.add_argument("--seq", type=int, default=None,

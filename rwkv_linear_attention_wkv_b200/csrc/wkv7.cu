@@ -9,12 +9,16 @@
 // The report gives no read-out; this library reads the state with the receptance as the
 // query, y_t = S_t r_t^T.
 //
-// One CTA per (batch row, head) of head size N = 64, 128 threads: thread pair (2i, 2i+1)
-// holds row i of S in registers, 32 columns each. The per-token vectors r, w, k, v, a, b
-// ([64] fp32 each) come in TMA tiles of kT7 tokens through a kS7-stage mbarrier pipeline;
-// y is staged in shared memory and TMA-stored a tile at a time. Per token and thread:
-// sa (32 FMA + one shuffle), the update (3 operations per element), y (32 FMA + one
-// shuffle). Bound: the FP32 pipe (about 5 N^2 operations per token per head).
+// One CTA per (batch row, head) of head size N = 64, 64 threads: thread t holds the 8 x 8
+// block of S at rows 8 (t / 8) .., columns {16 m + 2 (t mod 8), 16 m + 2 (t mod 8) + 1 : m < 4}
+// in registers. A token's vectors are read from shared memory once per thread (64-byte
+// contiguous, conflict-free 8-byte reads, shared by broadcast between row blocks) instead
+// of once per row, which keeps the shared-memory traffic per token at about 1.5 KB per
+// warp. Row sums (sa_i = S[i] . a and y_i = S[i] . r) reduce over the 8 threads of a row
+// block by recursive halving (7 shuffles for 8 rows), and sa is gathered back the same
+// way. r, w, k, v, a, b ([64] fp32 each per token) come in TMA tiles of kT7 tokens through
+// a kS7-stage mbarrier pipeline; y is staged in shared memory and TMA-stored a tile at a
+// time. Bound: the FP32 pipe (about 5 N^2 operations per token per head).
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
@@ -25,28 +29,63 @@ namespace {
 constexpr int kN7 = 64;        // head size
 constexpr int kT7 = 8;         // tokens per tile
 constexpr int kS7 = 4;         // pipeline stages
-constexpr int kHalf = kN7 / 2; // columns per thread
+constexpr int kBR = 8;         // rows of S per thread
+constexpr int kBC = 8;         // columns of S per thread (4 pairs, 16 columns apart)
+constexpr int kThr7 = (kN7 / kBR) * (kN7 / kBC);  // threads per head (64)
 constexpr int kTile7 = kT7 * kN7;  // floats per tensor tile
 
 struct Wkv7Maps {
   CUtensorMap r, w, k, v, a, b, y;
 };
 
-__global__ void __launch_bounds__(2 * kN7) wkv7_fwd_kernel(const __grid_constant__ Wkv7Maps maps,
-                                                          int B, int T, int H,
-                                                          const float* __restrict__ s0,
-                                                          float* __restrict__ s1,
-                                                          unsigned* err) {
+// Sum over the 8 lanes of a row block (lanes 8m .. 8m+7) of x[r] for each of the 8 rows:
+// recursive halving leaves lane l with the full sum for row (l mod 8).
+__device__ __forceinline__ float rowblock_reduce(float (&x)[kBR], int lc) {
+  // step 1: lanes differing in bit 2 exchange four rows
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const bool up = lc & 4;
+    const float send = up ? x[r] : x[r + 4];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
+    x[r] = (up ? x[r + 4] : x[r]) + got;  // now row r + 4 (up) or r (down)
+  }
+  // step 2: bit 1, two rows
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const bool up = lc & 2;
+    const float send = up ? x[r] : x[r + 2];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
+    x[r] = (up ? x[r + 2] : x[r]) + got;
+  }
+  // step 3: bit 0, one row
+  {
+    const bool up = lc & 1;
+    const float send = up ? x[0] : x[1];
+    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
+    x[0] = (up ? x[1] : x[0]) + got;
+  }
+  // lane lc holds row 4 (bit2) + 2 (bit1) + (bit0) = lc
+  return x[0];
+}
+
+__global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__ Wkv7Maps maps,
+                                                        int B, int T, int H,
+                                                        const float* __restrict__ s0,
+                                                        float* __restrict__ s1,
+                                                        unsigned* err) {
   // stage st: tiles r, w, k, v, a, b at smem + (6 st + slot) kTile7; y tiles after them
   extern __shared__ __align__(128) float smem7[];
   float* ybuf = smem7 + 6 * kS7 * kTile7;  // [2][kT7][64]
   __shared__ uint64_t bars[kS7];
   const int tid = threadIdx.x;
-  const int i = tid >> 1;            // row of S
-  const int c0 = (tid & 1) * kHalf;  // first column of this thread
+  const int lane = tid & 31;
+  const int lc = tid & 7;          // column block (and, after a row reduction, the row)
+  const int r0 = (tid >> 3) * kBR;  // first row of this thread's block
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh - b * H;
   const int ntile = (T + kT7 - 1) / kT7;
+  // column of pair m (0..3), element e (0..1) of this thread
+  auto col = [&](int m, int e) { return 16 * m + 2 * lc + e; };
 
   auto issue = [&](int st, int tile) {
     uint64_t* bar = &bars[st];
@@ -67,17 +106,18 @@ __global__ void __launch_bounds__(2 * kN7) wkv7_fwd_kernel(const __grid_constant
   }
   __syncthreads();
 
-  float S[kHalf];
+  float S[kBR][kBC];  // S[r][2m + e] = state[r0 + r][col(m, e)]
   {
-    const float* src = s0 ? s0 + (size_t(bh) * kN7 + i) * kN7 + c0 : nullptr;
+    const float* src = s0 ? s0 + (size_t(bh) * kN7 + r0) * kN7 : nullptr;
 #pragma unroll
-    for (int j = 0; j < kHalf; j += 4) {
-      const float4 q = src ? *reinterpret_cast<const float4*>(src + j) : make_float4(0, 0, 0, 0);
-      S[j] = q.x;
-      S[j + 1] = q.y;
-      S[j + 2] = q.z;
-      S[j + 3] = q.w;
-    }
+    for (int r = 0; r < kBR; ++r)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float2 x = src ? *reinterpret_cast<const float2*>(src + r * kN7 + col(m, 0))
+                             : make_float2(0.f, 0.f);
+        S[r][2 * m] = x.x;
+        S[r][2 * m + 1] = x.y;
+      }
   }
 
   for (int tile = 0; tile < ntile; ++tile) {
@@ -89,44 +129,58 @@ __global__ void __launch_bounds__(2 * kN7) wkv7_fwd_kernel(const __grid_constant
     __syncthreads();
     const int n = min(kT7, T - tile * kT7);
     for (int t = 0; t < n; ++t) {
-      const float* R = base + 0 * kTile7 + t * kN7 + c0;
-      const float* W = base + 1 * kTile7 + t * kN7 + c0;
-      const float* K = base + 2 * kTile7 + t * kN7 + c0;
-      const float vi = base[3 * kTile7 + t * kN7 + i];
-      const float* A = base + 4 * kTile7 + t * kN7 + c0;
-      const float* Bv = base + 5 * kTile7 + t * kN7 + c0;
-      // sa_i = S_{t-1}[i] . a_t, four partial sums for instruction-level parallelism
-      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+      const float* tok = base + t * kN7;
+      float wv[kBC], kv[kBC], av[kBC], bv[kBC], rv[kBC], vv[kBR];
 #pragma unroll
-      for (int j = 0; j < kHalf; j += 4) {
-        const float4 q = *reinterpret_cast<const float4*>(A + j);
-        p0 = fmaf(S[j], q.x, p0);
-        p1 = fmaf(S[j + 1], q.y, p1);
-        p2 = fmaf(S[j + 2], q.z, p2);
-        p3 = fmaf(S[j + 3], q.w, p3);
+      for (int m = 0; m < 4; ++m) {
+        const float2 rq = *reinterpret_cast<const float2*>(tok + 0 * kTile7 + col(m, 0));
+        const float2 wq = *reinterpret_cast<const float2*>(tok + 1 * kTile7 + col(m, 0));
+        const float2 kq = *reinterpret_cast<const float2*>(tok + 2 * kTile7 + col(m, 0));
+        const float2 aq = *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0));
+        const float2 bq = *reinterpret_cast<const float2*>(tok + 5 * kTile7 + col(m, 0));
+        rv[2 * m] = rq.x; rv[2 * m + 1] = rq.y;
+        wv[2 * m] = wq.x; wv[2 * m + 1] = wq.y;
+        kv[2 * m] = kq.x; kv[2 * m + 1] = kq.y;
+        av[2 * m] = aq.x; av[2 * m + 1] = aq.y;
+        bv[2 * m] = bq.x; bv[2 * m + 1] = bq.y;
       }
-      float sa = (p0 + p1) + (p2 + p3);
-      sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-      // S_t[i][j] = S[i][j] w_j + sa_i b_j + v_i k_j;  y_i = S_t[i] . r_t
-      float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+      {
+        const float4 v0 = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0);
+        const float4 v1 = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0 + 4);
+        vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
+        vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+      }
+      // sa_i = S_{t-1}[i] . a_t: partial sums over this thread's columns, then the row block
+      float part[kBR];
 #pragma unroll
-      for (int j = 0; j < kHalf; j += 4) {
-        const float4 wq = *reinterpret_cast<const float4*>(W + j);
-        const float4 kq = *reinterpret_cast<const float4*>(K + j);
-        const float4 bq = *reinterpret_cast<const float4*>(Bv + j);
-        const float4 rq = *reinterpret_cast<const float4*>(R + j);
-        S[j] = fmaf(S[j], wq.x, fmaf(sa, bq.x, vi * kq.x));
-        S[j + 1] = fmaf(S[j + 1], wq.y, fmaf(sa, bq.y, vi * kq.y));
-        S[j + 2] = fmaf(S[j + 2], wq.z, fmaf(sa, bq.z, vi * kq.z));
-        S[j + 3] = fmaf(S[j + 3], wq.w, fmaf(sa, bq.w, vi * kq.w));
-        y0 = fmaf(S[j], rq.x, y0);
-        y1 = fmaf(S[j + 1], rq.y, y1);
-        y2 = fmaf(S[j + 2], rq.z, y2);
-        y3 = fmaf(S[j + 3], rq.w, y3);
+      for (int r = 0; r < kBR; ++r) {
+        float p0 = S[r][0] * av[0], p1 = S[r][1] * av[1];
+#pragma unroll
+        for (int c = 2; c < kBC; c += 2) {
+          p0 = fmaf(S[r][c], av[c], p0);
+          p1 = fmaf(S[r][c + 1], av[c + 1], p1);
+        }
+        part[r] = p0 + p1;
       }
-      float yv = (y0 + y1) + (y2 + y3);
-      yv += __shfl_xor_sync(0xffffffffu, yv, 1);
-      if ((tid & 1) == 0) yt[t * kN7 + i] = yv;
+      const float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc
+      float sa[kBR];
+#pragma unroll
+      for (int r = 0; r < kBR; ++r) sa[r] = __shfl_sync(0xffffffffu, sa_mine, (lane & ~7) | r);
+      // S_t[i][j] = S[i][j] w_j + sa_i b_j + v_i k_j, then y_i = S_t[i] . r_t
+#pragma unroll
+      for (int r = 0; r < kBR; ++r) {
+        float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kBC; c += 2) {
+          S[r][c] = fmaf(S[r][c], wv[c], fmaf(sa[r], bv[c], vv[r] * kv[c]));
+          S[r][c + 1] = fmaf(S[r][c + 1], wv[c + 1], fmaf(sa[r], bv[c + 1], vv[r] * kv[c + 1]));
+          p0 = fmaf(S[r][c], rv[c], p0);
+          p1 = fmaf(S[r][c + 1], rv[c + 1], p1);
+        }
+        part[r] = p0 + p1;
+      }
+      const float y_mine = rowblock_reduce(part, lc);  // y for row r0 + lc
+      yt[t * kN7 + r0 + lc] = y_mine;
     }
     fence_proxy_async_smem();  // the y tile's writes, visible to the TMA store
     __syncthreads();           // the stage is consumed and the y tile complete
@@ -137,10 +191,12 @@ __global__ void __launch_bounds__(2 * kN7) wkv7_fwd_kernel(const __grid_constant
     }
   }
   if (s1 != nullptr) {
-    float* dst = s1 + (size_t(bh) * kN7 + i) * kN7 + c0;
+    float* dst = s1 + (size_t(bh) * kN7 + r0) * kN7;
 #pragma unroll
-    for (int j = 0; j < kHalf; j += 4)
-      *reinterpret_cast<float4*>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    for (int r = 0; r < kBR; ++r)
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        *reinterpret_cast<float2*>(dst + r * kN7 + col(m, 0)) = make_float2(S[r][2 * m], S[r][2 * m + 1]);
   }
   if (tid == 0) tma_store_wait_all();
 }
@@ -163,8 +219,8 @@ int launch_wkv7(int64_t B, int64_t T, int64_t H, const float* r, const float* w,
   if (cudaFuncSetAttribute(wkv7_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(smem)) != cudaSuccess)
     return WKV_ERR_CUDA;
-  wkv7_fwd_kernel<<<unsigned(B * H), 2 * kN7, smem, stream>>>(m, int(B), int(T), int(H), s0, s1,
-                                                              err);
+  wkv7_fwd_kernel<<<unsigned(B * H), kThr7, smem, stream>>>(m, int(B), int(T), int(H), s0, s1,
+                                                            err);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
