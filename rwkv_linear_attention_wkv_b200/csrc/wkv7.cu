@@ -11,7 +11,8 @@
 //
 // One CTA per (batch row, head) of head size N = 64, 64 threads: thread t holds the 8 x 8
 // block of S at rows 8 (t / 8) .., columns {16 m + 2 (t mod 8), 16 m + 2 (t mod 8) + 1 : m < 4}
-// in registers. A token's vectors are read from shared memory once per thread (64-byte
+// in registers, as pairs for packed fp32x2 arithmetic. A token's vectors are read from
+// shared memory once per thread (64-byte
 // contiguous, conflict-free 8-byte reads, shared by broadcast between row blocks) instead
 // of once per row, which keeps the shared-memory traffic per token at about 1.5 KB per
 // warp. Row sums (sa_i = S[i] . a and y_i = S[i] . r) reduce over the 8 threads of a row
@@ -38,33 +39,29 @@ struct Wkv7Maps {
   CUtensorMap r, w, k, v, a, b, y;
 };
 
-// Sum over the 8 lanes of a row block (lanes 8m .. 8m+7) of x[r] for each of the 8 rows:
-// recursive halving leaves lane l with the full sum for row (l mod 8).
+// Sum over the 8 lanes of a row block (lanes 8m .. 8m+7) of x[r] for each of the kBR rows:
+// recursive halving (exchange half the rows with the lane differing in bit 2, then bit 1,
+// ...) and, once one row is left, a butterfly sum. Lane l ends with the full sum for row
+// (l mod 8) >> (3 - log2 kBR) of the block.
 __device__ __forceinline__ float rowblock_reduce(float (&x)[kBR], int lc) {
-  // step 1: lanes differing in bit 2 exchange four rows
+  int half = kBR / 2;
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const bool up = lc & 4;
-    const float send = up ? x[r] : x[r + 4];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 4);
-    x[r] = (up ? x[r + 4] : x[r]) + got;  // now row r + 4 (up) or r (down)
-  }
-  // step 2: bit 1, two rows
+  for (int bit = 4; bit >= 1; bit >>= 1) {
+    if (half >= 1) {
+      const bool up = lc & bit;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const bool up = lc & 2;
-    const float send = up ? x[r] : x[r + 2];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 2);
-    x[r] = (up ? x[r + 2] : x[r]) + got;
+      for (int r = 0; r < kBR / 2; ++r) {
+        if (r < half) {
+          const float send = up ? x[r] : x[r + half];
+          const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+          x[r] = (up ? x[r + half] : x[r]) + got;
+        }
+      }
+      half >>= 1;
+    } else {
+      x[0] += __shfl_xor_sync(0xffffffffu, x[0], bit);
+    }
   }
-  // step 3: bit 0, one row
-  {
-    const bool up = lc & 1;
-    const float send = up ? x[0] : x[1];
-    const float got = __shfl_xor_sync(0xffffffffu, send, 1);
-    x[0] = (up ? x[1] : x[0]) + got;
-  }
-  // lane lc holds row 4 (bit2) + 2 (bit1) + (bit0) = lc
   return x[0];
 }
 
@@ -106,18 +103,15 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
   }
   __syncthreads();
 
-  float S[kBR][kBC];  // S[r][2m + e] = state[r0 + r][col(m, e)]
+  float2 S[kBR][kBC / 2];  // S[r][m] = state[r0 + r][col(m, 0 .. 1)]
   {
     const float* src = s0 ? s0 + (size_t(bh) * kN7 + r0) * kN7 : nullptr;
 #pragma unroll
     for (int r = 0; r < kBR; ++r)
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float2 x = src ? *reinterpret_cast<const float2*>(src + r * kN7 + col(m, 0))
-                             : make_float2(0.f, 0.f);
-        S[r][2 * m] = x.x;
-        S[r][2 * m + 1] = x.y;
-      }
+      for (int m = 0; m < 4; ++m)
+        S[r][m] = src ? *reinterpret_cast<const float2*>(src + r * kN7 + col(m, 0))
+                      : make_float2(0.f, 0.f);
   }
 
   for (int tile = 0; tile < ntile; ++tile) {
@@ -128,59 +122,52 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
     if (tile >= 2 && tid == 0) tma_store_wait_read<1>();  // this y buffer's last store has read it
     __syncthreads();
     const int n = min(kT7, T - tile * kT7);
+#pragma unroll 2
     for (int t = 0; t < n; ++t) {
       const float* tok = base + t * kN7;
-      float wv[kBC], kv[kBC], av[kBC], bv[kBC], rv[kBC], vv[kBR];
+      // the token's vectors at this thread's columns (pairs), and v at its rows
+      float2 rv[4], wv[4], kv[4], av[4], bv[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float2 rq = *reinterpret_cast<const float2*>(tok + 0 * kTile7 + col(m, 0));
-        const float2 wq = *reinterpret_cast<const float2*>(tok + 1 * kTile7 + col(m, 0));
-        const float2 kq = *reinterpret_cast<const float2*>(tok + 2 * kTile7 + col(m, 0));
-        const float2 aq = *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0));
-        const float2 bq = *reinterpret_cast<const float2*>(tok + 5 * kTile7 + col(m, 0));
-        rv[2 * m] = rq.x; rv[2 * m + 1] = rq.y;
-        wv[2 * m] = wq.x; wv[2 * m + 1] = wq.y;
-        kv[2 * m] = kq.x; kv[2 * m + 1] = kq.y;
-        av[2 * m] = aq.x; av[2 * m + 1] = aq.y;
-        bv[2 * m] = bq.x; bv[2 * m + 1] = bq.y;
+        rv[m] = *reinterpret_cast<const float2*>(tok + 0 * kTile7 + col(m, 0));
+        wv[m] = *reinterpret_cast<const float2*>(tok + 1 * kTile7 + col(m, 0));
+        kv[m] = *reinterpret_cast<const float2*>(tok + 2 * kTile7 + col(m, 0));
+        av[m] = *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0));
+        bv[m] = *reinterpret_cast<const float2*>(tok + 5 * kTile7 + col(m, 0));
       }
-      {
-        const float4 v0 = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0);
-        const float4 v1 = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0 + 4);
-        vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
-        vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+      float vv[kBR];
+#pragma unroll
+      for (int r = 0; r < kBR; r += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0 + r);
+        vv[r] = x.x; vv[r + 1] = x.y; vv[r + 2] = x.z; vv[r + 3] = x.w;
       }
-      // sa_i = S_{t-1}[i] . a_t: partial sums over this thread's columns, then the row block
+      // sa_i = S_{t-1}[i] . a_t: partial sums over this thread's columns (packed fp32x2
+      // multiply-adds), then over the row block
       float part[kBR];
 #pragma unroll
       for (int r = 0; r < kBR; ++r) {
-        float p0 = S[r][0] * av[0], p1 = S[r][1] * av[1];
+        float2 p = __fmul2_rn(S[r][0], av[0]);
 #pragma unroll
-        for (int c = 2; c < kBC; c += 2) {
-          p0 = fmaf(S[r][c], av[c], p0);
-          p1 = fmaf(S[r][c + 1], av[c + 1], p1);
-        }
-        part[r] = p0 + p1;
+        for (int m = 1; m < 4; ++m) p = __ffma2_rn(S[r][m], av[m], p);
+        part[r] = p.x + p.y;
       }
-      const float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc
-      float sa[kBR];
-#pragma unroll
-      for (int r = 0; r < kBR; ++r) sa[r] = __shfl_sync(0xffffffffu, sa_mine, (lane & ~7) | r);
+      const float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc / (8 / kBR)
       // S_t[i][j] = S[i][j] w_j + sa_i b_j + v_i k_j, then y_i = S_t[i] . r_t
 #pragma unroll
       for (int r = 0; r < kBR; ++r) {
-        float p0 = 0.f, p1 = 0.f;
+        const float sr = __shfl_sync(0xffffffffu, sa_mine, (lane & ~7) | (r * (8 / kBR)));
+        const float2 sa2 = make_float2(sr, sr);
+        const float2 v2 = make_float2(vv[r], vv[r]);
+        float2 p = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < kBC; c += 2) {
-          S[r][c] = fmaf(S[r][c], wv[c], fmaf(sa[r], bv[c], vv[r] * kv[c]));
-          S[r][c + 1] = fmaf(S[r][c + 1], wv[c + 1], fmaf(sa[r], bv[c + 1], vv[r] * kv[c + 1]));
-          p0 = fmaf(S[r][c], rv[c], p0);
-          p1 = fmaf(S[r][c + 1], rv[c + 1], p1);
+        for (int m = 0; m < 4; ++m) {
+          S[r][m] = __ffma2_rn(S[r][m], wv[m], __ffma2_rn(sa2, bv[m], __fmul2_rn(v2, kv[m])));
+          p = __ffma2_rn(S[r][m], rv[m], p);
         }
-        part[r] = p0 + p1;
+        part[r] = p.x + p.y;
       }
-      const float y_mine = rowblock_reduce(part, lc);  // y for row r0 + lc
-      yt[t * kN7 + r0 + lc] = y_mine;
+      const float y_mine = rowblock_reduce(part, lc);  // y for row r0 + lc / (8 / kBR)
+      if (lc % (8 / kBR) == 0) yt[t * kN7 + r0 + lc / (8 / kBR)] = y_mine;
     }
     fence_proxy_async_smem();  // the y tile's writes, visible to the TMA store
     __syncthreads();           // the stage is consumed and the y tile complete
@@ -195,8 +182,7 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
 #pragma unroll
     for (int r = 0; r < kBR; ++r)
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
-        *reinterpret_cast<float2*>(dst + r * kN7 + col(m, 0)) = make_float2(S[r][2 * m], S[r][2 * m + 1]);
+      for (int m = 0; m < 4; ++m) *reinterpret_cast<float2*>(dst + r * kN7 + col(m, 0)) = S[r][m];
   }
   if (tid == 0) tma_store_wait_all();
 }
