@@ -33,6 +33,17 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
                                       const void* r, void* y, int bf16, cudaStream_t stream);
 
 /*
+ * Runs the backward on a small internal problem (B = 1, T = 192, C = 32: three segments
+ * of the time-parallel reverse pass; every input zero) in which the last segment
+ * withholds its published map, so the earlier segments wait for a flag that nothing sets
+ * and give up after `wait_ns` nanoseconds (bounded wait; no trap, no hang). The kernels
+ * still end and the next wkv_stream_status(stream) returns WKV_ERR_TIMEOUT, after which
+ * the error word is clear again. Allocates its buffers with cudaMallocAsync on `stream`
+ * and frees them in stream order. Returns the launch status.
+ */
+WKV_API int wkv_testing_backward_timeout(uint64_t wait_ns, cudaStream_t stream);
+
+/*
  * Forces the backward's plain (non-TMA) tile movement; otherwise as wkv_backward.
  */
 WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const float* w,

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m rwkv_linear_attention_wkv_b200.build`"
+        f"{LIB_PATH} is missing: build it with `python rwkv_linear_attention_wkv_b200/build.py`"
         " (the WKV operator has no non-CUDA implementation)")
 
 lib = ctypes.CDLL(LIB_PATH)
@@ -44,10 +44,15 @@ _SIGS = {
     "wkv_testing_backward_state_plain": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
                                          ctypes.c_int),
     "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
+    "wkv_testing_backward_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
     "wkv_testing_forward_plain": ([_I, _I, _I] + [_P] * 6 + [ctypes.c_int, _P], ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
-    _f = getattr(lib, _name)
+    try:
+        _f = getattr(lib, _name)
+    except AttributeError as _e:
+        raise ImportError(f"{LIB_PATH} lacks {_name}: it is older than the sources; rebuild it "
+                          "with `python rwkv_linear_attention_wkv_b200/build.py`") from _e
     _f.argtypes = _args
     _f.restype = _res
 

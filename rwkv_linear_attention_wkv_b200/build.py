@@ -1,6 +1,9 @@
 """Builds libwkv.so (the CUDA library behind include/wkv.h) in this package directory.
 
-    python -m rwkv_linear_attention_wkv_b200.build [--verbose-ptxas]
+    python rwkv_linear_attention_wkv_b200/build.py [--verbose-ptxas] [--force]
+
+(Run as a script, or load this file by path: importing it as a submodule would first
+import the package, which needs the library this builds.)
 
 nvcc compiles every csrc/*.cu for sm_100a only and links one shared library with the
 CUDA runtime linked statically, so loading it needs no GPU and no torch.

@@ -11,6 +11,8 @@
 
 namespace wkv {
 
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
 // Device error word (one per device context): bit kErrTimeout is set by a kernel that
 // gave up a bounded wait. Read and cleared by wkv_stream_status().
 __device__ unsigned g_error_word;
@@ -336,6 +338,40 @@ WKV_API int wkv_testing_lookback_timeout(uint64_t wait_ns, cudaStream_t stream) 
   if (rc == WKV_OK) {
     FwdArgs a{B, T, C, w, u, k, v, r, y, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, err};
     rc = launch_fwd_chunked_ex(a, ws, nseg, (unsigned long long)wait_ns, 1, stream);
+  }
+  cudaFreeAsync(buf, stream);
+  return rc;
+}
+
+WKV_API int wkv_testing_backward_timeout(uint64_t wait_ns, cudaStream_t stream) {
+  const int64_t B = 1, T = 192, C = 32;  // 12 chunks of 16 tokens: 3 reverse segments
+  const size_t n = align_up(size_t(B * T * C) * sizeof(float), 256);
+  const size_t c4 = align_up(size_t(C) * sizeof(float), 256);
+  const size_t wsb = backward_workspace_bytes(B, T, C);
+  const size_t total = 7 * n + 4 * c4 + wsb + 256;
+  char* buf = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&buf), total, stream) != cudaSuccess)
+    return WKV_ERR_CUDA;
+  if (cudaMemsetAsync(buf, 0, total, stream) != cudaSuccess) {
+    cudaFreeAsync(buf, stream);
+    return WKV_ERR_CUDA;
+  }
+  char* p = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(buf) + 255) & ~uintptr_t(255));
+  auto take = [&](size_t bytes) {
+    float* q = reinterpret_cast<float*>(p);
+    p += bytes;
+    return q;
+  };
+  float *k = take(n), *v = take(n), *r = take(n), *dy = take(n), *dk = take(n), *dv = take(n),
+        *dr = take(n), *w = take(c4), *u = take(c4), *dw = take(c4), *du = take(c4);
+  void* ws = p;
+  unsigned* err = error_word();
+  int rc = err ? WKV_OK : WKV_ERR_CUDA;
+  if (rc == WKV_OK) {
+    BwdArgs a{B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, ws, err};
+    a.wait_ns = (unsigned long long)wait_ns;
+    a.withhold_last_map = 1;
+    rc = launch_backward(a, false, stream);
   }
   cudaFreeAsync(buf, stream);
   return rc;

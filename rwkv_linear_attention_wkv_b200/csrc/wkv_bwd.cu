@@ -363,7 +363,7 @@ __device__ __forceinline__ Agg chunk_aggregate(const float* K, const float* V, i
 
 __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
     const __grid_constant__ TensorMaps4 maps, int B, int T, int C, const float* __restrict__ w,
-    const StateIO io, void* ws, unsigned* err) {
+    const StateIO io, void* ws, unsigned* err, unsigned long long wait_ns) {
   constexpr int kTile = kTT * 32;
   constexpr int kSegC = kSW * kCK;  // chunks per checkpoint segment
   __shared__ __align__(128) float tiles[kSW][kCK][2][kTile];  // k, v of each warp's chunks
@@ -467,7 +467,7 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
       cp_async_wait_all();
     } else {  // wait for the flags not yet set, then fetch (L2 loads: L1 may be stale)
       const unsigned* flag = lane < m ? &lay.fflags[item0 + j0 + lane] : &lay.fflags[item0 + j0];
-      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, kWaitLimitNs, err) : 1u;
+      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, wait_ns, err) : 1u;
       ok = __all_sync(0xffffffffu, fl != 0);
       __syncwarp();  // orders every lane's acquire before every lane's fetch below
       if (ok) {  // (a wait that gave up flagged the error word: continue from the empty state)
@@ -880,7 +880,8 @@ __global__ void __launch_bounds__(kSW * 32, 5)
     wkv_bwd_seg_kernel(const __grid_constant__ TensorMaps4 in_maps,
                        const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
                        const float* __restrict__ w, const float* __restrict__ u,
-                       const StateIO io, void* ws, unsigned* err) {
+                       const StateIO io, void* ws, unsigned* err, unsigned long long wait_ns,
+                       int withhold_last_map) {
   constexpr int kTile = kTT * 32;
   constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
   // Dynamic: [kSW warps][kNL tiles][kTile] floats.
@@ -998,7 +999,8 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   __syncthreads();
 
   // ---- 2. the segment's map; the carry at its end ----
-  if (warp == 0 && seg > 0) {  // the segment's map, for the segments before it
+  if (warp == 0 && seg > 0 && !(withhold_last_map && seg == nseg - 1)) {
+    // the segment's map, for the segments before it
     RevAgg M = get_agg(sagg[kSW - 1][lane][0], sagg[kSW - 1][lane][1]);
 #pragma unroll
     for (int i = kSW - 2; i >= 0; --i) M = rev_compose(get_agg(sagg[i][lane][0], sagg[i][lane][1]), M);
@@ -1012,7 +1014,7 @@ __global__ void __launch_bounds__(kSW * 32, 5)
       cp_async_wait_all();
     } else {  // wait for the flags not yet set, then fetch (L2 loads: L1 may be stale)
       const unsigned* flag = lane < m ? &lay.rflags[item0 + seg + 1 + lane] : &lay.rflags[item0 + jc];
-      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, kWaitLimitNs, err) : 1u;
+      const unsigned fl = fwant != 0 ? wait_flag(flag, fwant, wait_ns, err) : 1u;
       ok = __all_sync(0xffffffffu, fl != 0);
       __syncwarp();  // orders every lane's acquire before every lane's fetch below
       if (ok) {  // (a wait that gave up flagged the error word: continue from a zero carry)
@@ -1154,7 +1156,8 @@ int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, 
       cudaSuccess)
     return WKV_ERR_CUDA;
   kern<<<unsigned(nitems), kSW * 32, smem, stream>>>(in, out, int(a.B), int(a.T), int(a.C), a.w,
-                                                      a.u, state_io(a), a.ws, a.err);
+                                                      a.u, state_io(a), a.ws, a.err, a.wait_ns,
+                                                      a.withhold_last_map);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -1183,7 +1186,7 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     const int64_t nch = (a.T + kTT - 1) / kTT;
     const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
     wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
-        ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err);
+        ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
     if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     if (a.r)
       rc = a.dr ? launch_seg<true, true>(a, in, out, nitems, stream)

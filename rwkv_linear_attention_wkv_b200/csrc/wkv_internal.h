@@ -100,6 +100,10 @@ struct BwdArgs {
   float* da0 = nullptr;
   float* db0 = nullptr;
   float* dp0 = nullptr;
+  // Chain waits of the time-parallel passes: their limit (ns) and, for tests of the
+  // bounded wait only, the last segment of the reverse pass withholding its published map.
+  unsigned long long wait_ns = 2000000000ull;
+  int withhold_last_map = 0;
 };
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);

@@ -114,3 +114,16 @@ def test_backward_workspace_checks(W):
     z = torch.zeros((1, 0, 8), device="cuda")
     g = W.wkv_backward(dev(x.w), dev(x.u), z, z, z, z)
     assert torch.count_nonzero(g["dw"]) == 0 and torch.count_nonzero(g["du"]) == 0
+
+
+def test_backward_wait_gives_up_and_reports(W):
+    # The last segment of the time-parallel reverse pass withholds its map: the earlier
+    # segments' bounded waits give up after 1 ms, flag the error word and end.
+    import ctypes
+    s = torch.cuda.current_stream()
+    rc = W.lib.wkv_testing_backward_timeout(1_000_000, ctypes.c_void_p(s.cuda_stream))
+    assert rc == 0
+    assert W.wkv_stream_status() == 4          # WKV_ERR_TIMEOUT
+    assert W.wkv_stream_status() == 0          # cleared
+    x = wkv_inputs.make_inputs(1, 200, 32, seed=21, with_dy=True)  # context still usable
+    check(W, x)
