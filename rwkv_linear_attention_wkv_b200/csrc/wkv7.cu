@@ -65,6 +65,35 @@ __device__ __forceinline__ float rowblock_reduce(float (&x)[kBR], int lc) {
   return x[0];
 }
 
+// Two row reductions at once (independent shuffles interleave).
+__device__ __forceinline__ void rowblock_reduce2(float (&x)[kBR], float (&z)[kBR], int lc,
+                                                 float& xs, float& zs) {
+  int half = kBR / 2;
+#pragma unroll
+  for (int bit = 4; bit >= 1; bit >>= 1) {
+    if (half >= 1) {
+      const bool up = lc & bit;
+#pragma unroll
+      for (int r = 0; r < kBR / 2; ++r) {
+        if (r < half) {
+          const float sx = up ? x[r] : x[r + half];
+          const float sz = up ? z[r] : z[r + half];
+          const float gx = __shfl_xor_sync(0xffffffffu, sx, bit);
+          const float gz = __shfl_xor_sync(0xffffffffu, sz, bit);
+          x[r] = (up ? x[r + half] : x[r]) + gx;
+          z[r] = (up ? z[r + half] : z[r]) + gz;
+        }
+      }
+      half >>= 1;
+    } else {
+      x[0] += __shfl_xor_sync(0xffffffffu, x[0], bit);
+      z[0] += __shfl_xor_sync(0xffffffffu, z[0], bit);
+    }
+  }
+  xs = x[0];
+  zs = z[0];
+}
+
 __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__ Wkv7Maps maps,
                                                         int B, int T, int H,
                                                         const float* __restrict__ s0,
@@ -122,18 +151,37 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
     if (tile >= 2 && tid == 0) tma_store_wait_read<1>();  // this y buffer's last store has read it
     __syncthreads();
     const int n = min(kT7, T - tile * kT7);
-#pragma unroll 2
+    // sa for the tile's first token: S_{t-1} . a_t summed over this thread's columns, then
+    // over the row block. Within the tile the next token's sa is computed together with
+    // this token's y (both read the updated state), so their two row reductions run
+    // side by side.
+    float part[kBR], part2[kBR];
+    {
+      const float* tok = base;
+#pragma unroll
+      for (int r = 0; r < kBR; ++r) {
+        float2 p = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m)
+          p = __ffma2_rn(S[r][m], *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0)), p);
+        part[r] = p.x + p.y;
+      }
+    }
+    float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc / (8 / kBR)
+#pragma unroll 1
     for (int t = 0; t < n; ++t) {
       const float* tok = base + t * kN7;
+      const bool next = t + 1 < n;
       // the token's vectors at this thread's columns (pairs), and v at its rows
-      float2 rv[4], wv[4], kv[4], av[4], bv[4];
+      float2 rv[4], wv[4], kv[4], bv[4], an[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         rv[m] = *reinterpret_cast<const float2*>(tok + 0 * kTile7 + col(m, 0));
         wv[m] = *reinterpret_cast<const float2*>(tok + 1 * kTile7 + col(m, 0));
         kv[m] = *reinterpret_cast<const float2*>(tok + 2 * kTile7 + col(m, 0));
-        av[m] = *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0));
         bv[m] = *reinterpret_cast<const float2*>(tok + 5 * kTile7 + col(m, 0));
+        an[m] = next ? *reinterpret_cast<const float2*>(tok + kN7 + 4 * kTile7 + col(m, 0))
+                     : make_float2(0.f, 0.f);  // a of the next token
       }
       float vv[kBR];
 #pragma unroll
@@ -141,32 +189,29 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
         const float4 x = *reinterpret_cast<const float4*>(tok + 3 * kTile7 + r0 + r);
         vv[r] = x.x; vv[r + 1] = x.y; vv[r + 2] = x.z; vv[r + 3] = x.w;
       }
-      // sa_i = S_{t-1}[i] . a_t: partial sums over this thread's columns (packed fp32x2
-      // multiply-adds), then over the row block
-      float part[kBR];
-#pragma unroll
-      for (int r = 0; r < kBR; ++r) {
-        float2 p = __fmul2_rn(S[r][0], av[0]);
-#pragma unroll
-        for (int m = 1; m < 4; ++m) p = __ffma2_rn(S[r][m], av[m], p);
-        part[r] = p.x + p.y;
-      }
-      const float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc / (8 / kBR)
-      // S_t[i][j] = S[i][j] w_j + sa_i b_j + v_i k_j, then y_i = S_t[i] . r_t
+      // S_t[i][j] = S[i][j] w_j + sa_i b_j + v_i k_j; then y_i = S_t[i] . r_t and the next
+      // token's sa_i = S_t[i] . a_{t+1}
 #pragma unroll
       for (int r = 0; r < kBR; ++r) {
         const float sr = __shfl_sync(0xffffffffu, sa_mine, (lane & ~7) | (r * (8 / kBR)));
         const float2 sa2 = make_float2(sr, sr);
         const float2 v2 = make_float2(vv[r], vv[r]);
-        float2 p = make_float2(0.f, 0.f);
+        float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           S[r][m] = __ffma2_rn(S[r][m], wv[m], __ffma2_rn(sa2, bv[m], __fmul2_rn(v2, kv[m])));
           p = __ffma2_rn(S[r][m], rv[m], p);
+          q = __ffma2_rn(S[r][m], an[m], q);
         }
         part[r] = p.x + p.y;
+        part2[r] = q.x + q.y;
       }
-      const float y_mine = rowblock_reduce(part, lc);  // y for row r0 + lc / (8 / kBR)
+      float y_mine;
+      if (next) {
+        rowblock_reduce2(part, part2, lc, y_mine, sa_mine);
+      } else {
+        y_mine = rowblock_reduce(part, lc);
+      }
       if (lc % (8 / kBR) == 0) yt[t * kN7 + r0 + lc / (8 / kBR)] = y_mine;
     }
     fence_proxy_async_smem();  // the y tile's writes, visible to the TMA store
