@@ -41,6 +41,7 @@
 #include <algorithm>
 
 #include "wkv_internal.h"
+#include "wkv_async.cuh"
 #include "wkv_step.cuh"
 
 namespace wkv {

@@ -183,14 +183,6 @@ __device__ __forceinline__ void tma_store_wait_all() {
 }
 
 // Generic-proxy writes to shared memory become visible to the async proxy (TMA store).
-// 16-byte asynchronous copy global -> shared through L2 only (cp.async.cg), and its wait.
-__device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

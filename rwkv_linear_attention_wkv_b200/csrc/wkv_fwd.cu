@@ -27,9 +27,22 @@ namespace wkv {
 // window first, then the log-weights and their running max, then the per-token
 // arithmetic, then every store. (Token by token, each token's loads would wait for the
 // previous token's store, which the compiler must assume may alias them.)
+//
+// In the single-exponential output form, windows of two or more tokens go through
+// window_fast_pairs: the same operations with the ones that do not lie on the recurrence's
+// serial chains packed two tokens to an fp32x2 instruction.
+template <typename Tin, bool GATE, int RB, int RS>
+__device__ __forceinline__ void window_fast_pairs(ChanState& s, const ChanParams& cp,
+                                                  const Tin* K, const Tin* V, const Tin* R,
+                                                  Tin* Y);
+
 template <typename Tin, bool GATE, bool FASTOUT, int RB, int RS>
 __device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, const Tin* K,
                                             const Tin* V, const Tin* R, Tin* Y) {
+  if constexpr (FASTOUT && RB >= 2) {
+    window_fast_pairs<Tin, GATE, RB, RS>(s, cp, K, V, R, Y);
+    return;
+  }
   float kk[RB], vv[RB], m[RB], d[RB], den[RB], num[RB];
   float rr[GATE ? RB : 1];
 #pragma unroll
@@ -86,6 +99,94 @@ __device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, 
 #pragma unroll
   for (int j = 0; j < RB; ++j)
     Y[j * RS] = Elem<Tin>::from_f(FASTOUT ? num[j] * rcp(den[j]) : num[j]);
+  wkv_rebase(s, float(RB) * cp.w2);
+}
+
+// Tokens 2i and 2i+1 of the window share an fp32x2 register pair for every quantity that is
+// not on a serial chain: log-weights, their differences from the running maximum, the
+// selected factors, products with v and H, numerator, denominator, output. The chains
+// themselves (running maximum Q, a, b) stay scalar, token by token, and the value of a (b)
+// before each token lands in its half of a pair for the output's fma. Each packed
+// instruction rounds its lanes as the scalar form would, so the results are those of the
+// scalar code bit for bit.
+template <typename Tin, bool GATE, int RB, int RS>
+__device__ __forceinline__ void window_fast_pairs(ChanState& s, const ChanParams& cp,
+                                                  const Tin* K, const Tin* V, const Tin* R,
+                                                  Tin* Y) {
+  static_assert(RB % 2 == 0, "token pairs");
+  constexpr int NP = RB / 2;
+  float2 kk[NP], vv[NP], rr[GATE ? NP : 1];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    kk[i] = make_float2(Elem<Tin>::to_f(K[2 * i * RS]), Elem<Tin>::to_f(K[(2 * i + 1) * RS]));
+    vv[i] = make_float2(Elem<Tin>::to_f(V[2 * i * RS]), Elem<Tin>::to_f(V[(2 * i + 1) * RS]));
+    if (GATE)
+      rr[i] = make_float2(Elem<Tin>::to_f(R[2 * i * RS]), Elem<Tin>::to_f(R[(2 * i + 1) * RS]));
+  }
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const float2 w2 = make_float2(cp.w2, cp.w2);
+  const float2 npl = make_float2(-s.pl, -s.pl);
+  float2 m[NP], d[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+    m[i] = __ffma2_rn(make_float2(float(2 * i + 1), float(2 * i + 2)), w2,
+                      __ffma2_rn(kk[i], l2e, npl));
+  float Q = s.Q;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    float2 qp;  // the running maximum before each token of the pair
+    qp.x = Q;
+    Q = fmaxf(Q, m[i].x);
+    qp.y = Q;
+    Q = fmaxf(Q, m[i].y);
+    d[i] = __ffma2_rn(qp, make_float2(-1.f, -1.f), m[i]);  // m - Q, one rounding
+  }
+  s.Q = Q;
+  float2 e1[NP], e2[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const float ex = ex2(-fabsf(d[i].x)), ey = ex2(-fabsf(d[i].y));
+    const bool cx = d[i].x > 0.f, cy = d[i].y > 0.f;
+    e1[i] = make_float2(cx ? ex : 1.f, cy ? ey : 1.f);
+    e2[i] = make_float2(cx ? 1.f : ex, cy ? 1.f : ey);
+  }
+  float2 er[GATE ? NP : 1];
+  if (GATE) {
+    const float2 nl2e = make_float2(-kLog2e, -kLog2e);
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const float2 x = __fmul2_rn(rr[i], nl2e);
+      er[i] = make_float2(ex2(x.x), ex2(x.y));
+    }
+  }
+  const float2 H = make_float2(cp.H, cp.H);
+  float a = s.a, b = s.b;
+  float2 num[NP], den[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const float2 ev = __fmul2_rn(e2[i], vv[i]);
+    const float2 he = __fmul2_rn(H, e2[i]);
+    float2 ap, bp;  // a and b before each token of the pair
+    ap.x = a;
+    bp.x = b;
+    a = fmaf(e1[i].x, a, ev.x);
+    b = fmaf(e1[i].x, b, e2[i].x);
+    ap.y = a;
+    bp.y = b;
+    a = fmaf(e1[i].y, a, ev.y);
+    b = fmaf(e1[i].y, b, e2[i].y);
+    num[i] = __ffma2_rn(e1[i], ap, __fmul2_rn(he, vv[i]));
+    den[i] = __ffma2_rn(e1[i], bp, he);
+    if (GATE) den[i] = __ffma2_rn(den[i], er[i], den[i]);
+  }
+  s.a = a;
+  s.b = b;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const float2 y = __fmul2_rn(num[i], make_float2(rcp(den[i].x), rcp(den[i].y)));
+    Y[2 * i * RS] = Elem<Tin>::from_f(y.x);
+    Y[(2 * i + 1) * RS] = Elem<Tin>::from_f(y.y);
+  }
   wkv_rebase(s, float(RB) * cp.w2);
 }
 

@@ -27,6 +27,7 @@
 // Every wait is bounded in wall time; a wait that gives up flags the error word and
 // carries on with an empty carry (the result is then wrong, but the kernel ends).
 #include "wkv_internal.h"
+#include "wkv_async.cuh"
 #include "wkv_step.cuh"
 
 namespace wkv {

@@ -101,6 +101,40 @@ def test_bf16_streaming_kernel_matches_plain_kernel_bitwise(W, shape):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+def run_bf16(W, x, plain=False):
+    import ctypes
+    w, u = dev(x.w), dev(x.u)
+    k, v, r = (dev_bf16(x.bits[n]) for n in "kvr")
+    if not plain:
+        y = W.wkv_forward_bf16(w, u, k, v, r)
+    else:
+        y = torch.empty_like(k)
+        P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        rc = W.lib.wkv_testing_forward_plain(x.B, x.T, x.C, P(w), P(u), P(k), P(v), P(r), P(y),
+                                             1, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert rc == 0, W.wkv_status_string(rc)
+    assert W.wkv_stream_status() == 0
+    return host_bf16(y)
+
+
+@pytest.mark.parametrize("plain", [False, True])
+def test_bf16_gate_extremes(W, plain):
+    # Receptances far into both saturated ends of the gate (|r| up to 150), and a NaN
+    # receptance, which must give a NaN output there and nowhere else.
+    B, T, C = 2, 96, 128
+    x = wkv_inputs.make_inputs(B, T, C, seed=24, dtype="bf16", k_std=2.0)
+    g = np.random.Generator(np.random.PCG64(25))
+    r = g.uniform(-150.0, 150.0, (B, T, C)).astype(np.float32)
+    r[:, ::7] = g.uniform(-4.0, 4.0, (B, (T + 6) // 7, C))
+    x.bits["r"] = wkv_inputs.round_to_bf16_bits(r)
+    x.r = wkv_inputs.bf16_bits_to_f32(x.bits["r"])
+    ref = oracle.wkv_recurrent(x.w, x.u, x.k, x.v, x.r)
+    assert_bf16_close(run_bf16(W, x, plain), ref)
+    x.bits["r"][1, 40, 77] = 0x7FC0  # bf16 NaN
+    nan = np.isnan(run_bf16(W, x, plain))
+    assert nan[1, 40, 77] and nan.sum() == 1
+
+
 def test_single_token_is_v_and_constant_v(W):
     x = wkv_inputs.make_inputs(3, 1, 64, seed=3, k_std=5.0)
     y = run_f32(W, x, gate=False)
