@@ -37,6 +37,7 @@ BYTES_PER_ELEM = 8          # read k, v, r and write y, 2 bytes each
 FALLBACK_HBM_GBS = 6650.0
 KERNEL = "wkv_fwd_tma_kernel<bf16, gate=1, TT=32, S=3, NW=1>"
 KERNEL_SOURCES = ["rwkv_linear_attention_wkv_b200/csrc/wkv_fwd.cu",
+                  "rwkv_linear_attention_wkv_b200/csrc/wkv_window.cuh",
                   "rwkv_linear_attention_wkv_b200/csrc/wkv_step.cuh",
                   "rwkv_linear_attention_wkv_b200/csrc/wkv_device.cuh"]
 TRAFFIC_FILE = "profiles/wkv_fwd_tma_bf16__B8_T4096_C4096.md"

@@ -15,7 +15,8 @@
 // a CTA waits for belongs to a CTA that started earlier. Single pass, 16 bytes of HBM
 // traffic per element:
 //   1. every warp TMA-loads its k, v, r sub-tile into shared memory (kept resident) and
-//      folds k, v into the sub-chunk aggregate from the empty state;
+//      folds k, v into the sub-chunk aggregate from the empty state (whole sub-chunks in
+//      windows, as the streaming kernel runs them);
 //   2. warp 0 combines the W aggregates and publishes the segment's aggregate; the last
 //      warp forms the state entering the segment in a fixed order from the published
 //      aggregates of up to kFold earlier segments and the state entering the first of
@@ -29,6 +30,7 @@
 #include "wkv_internal.h"
 #include "wkv_async.cuh"
 #include "wkv_step.cuh"
+#include "wkv_window.cuh"
 
 namespace wkv {
 
@@ -36,11 +38,11 @@ namespace {
 
 // Segment shape (the macros exist for sweeps): kW warps per CTA, each owning a sub-chunk
 // of kLS tokens; and the channel count below which the time-parallel path is used. The
-// streaming kernel runs each channel's tokens at its per-warp latency (about 30 ns a token
-// on B200), this kernel at about 4.5 ps an element over the whole GPU: below ~8192
-// channels (256 warps, 1.7 per SM) the time-parallel path is faster (measured: 16 x 1024 x
-// 768 streams in 37 us against 80 us chunked; 1 x 32768 x 4096 chunked in 0.60 ms against
-// 0.94 ms streaming).
+// streaming kernel runs each channel's tokens at its per-warp latency (about 29 ns a token
+// on B200: one warp walks 4096 tokens in 119 us), this kernel at about 3.4 ps an element
+// over the whole GPU (1 x 32768 x 4096 in 0.45 ms, against 0.94 ms streaming): the two
+// cross near 29 ns / 3.4 ps = 8500 channels, so below 8192 channels (256 warps, 1.7 per
+// SM) the time-parallel path is taken.
 #ifndef WKV_SCAN_W
 #define WKV_SCAN_W 8
 #endif
@@ -164,7 +166,9 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   if (n > 0) mbar_wait(bar, 0, err);
   __syncwarp();
   ChanState s = empty_state();
-  {
+  if (n == kLS) {
+    absorb_full_tile<kLS, 32>(s, cp, K, V, rb);
+  } else {
     int j = 0;
     for (int t = 0; t < n; ++t) {
       wkv_absorb(s, cp, float(j + 1), K[t * 32], V[t * 32]);
@@ -237,17 +241,24 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   s = to_state(cin);
   if (n > 0) {
     const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
-    int j = 0;
-    for (int t = 0; t < n; ++t) {
-      const float kk = K[t * 32], vv = V[t * 32], rr = GATE ? R[t * 32] : 0.f;
-      Y[t * 32] = fast ? wkv_token<GATE, true>(s, cp, float(j + 1), kk, vv, rr)
-                       : wkv_token<GATE, false>(s, cp, float(j + 1), kk, vv, rr);
-      if (++j == rb) {
-        wkv_rebase(s, float(rb) * cp.w2);
-        j = 0;
+    if (n == kLS) {  // whole windows (y overwrites k only after the window has read it)
+      if (fast)
+        full_tile<float, GATE, true, kLS, 32>(s, cp, K, V, R, Y, rb);
+      else
+        full_tile<float, GATE, false, kLS, 32>(s, cp, K, V, R, Y, rb);
+    } else {
+      int j = 0;
+      for (int t = 0; t < n; ++t) {
+        const float kk = K[t * 32], vv = V[t * 32], rr = GATE ? R[t * 32] : 0.f;
+        Y[t * 32] = fast ? wkv_token<GATE, true>(s, cp, float(j + 1), kk, vv, rr)
+                         : wkv_token<GATE, false>(s, cp, float(j + 1), kk, vv, rr);
+        if (++j == rb) {
+          wkv_rebase(s, float(rb) * cp.w2);
+          j = 0;
+        }
       }
+      if (j) wkv_rebase_partial(s, j, cp.w2);
     }
-    if (j) wkv_rebase_partial(s, j, cp.w2);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
