@@ -343,10 +343,34 @@ __device__ __forceinline__ Agg chunk_aggregate(const float* K, const float* V, i
                                                const ChanParams& cp) {
   ChanState s = empty_state();
   if (n == kTT) {
+    // absorb_indep token by token, with the log-weights and the products e2 v two tokens
+    // to an fp32x2 instruction (each lane rounded as the scalar form)
+    const float2 l2e = make_float2(kLog2e, kLog2e);
+    const float2 w2 = make_float2(cp.w2, cp.w2);
 #pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      absorb_indep(s, cp, float(t % RB + 1), K[t * 32], V[t * 32]);
-      if ((t + 1) % RB == 0) wkv_rebase(s, float(RB) * cp.w2);
+    for (int t = 0; t < kTT; t += 2) {
+      const float2 kk = make_float2(K[t * 32], K[(t + 1) * 32]);
+      const float2 vv = make_float2(V[t * 32], V[(t + 1) * 32]);
+      const float2 m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
+                                  __fmul2_rn(kk, l2e));
+      float e1s[2], e2s[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float mh = h ? m.y : m.x;
+        const float d = (mh - s.Q) - s.pl;
+        const float e = ex2(-fabsf(d));
+        const bool c = d > 0.f;
+        e1s[h] = c ? e : 1.f;
+        e2s[h] = c ? 1.f : e;
+        s.Q = c ? mh : s.Q;
+        s.pl = c ? 0.f : s.pl;
+        if ((t + h + 1) % RB == 0) wkv_rebase(s, float(RB) * cp.w2);
+      }
+      const float2 ev = __fmul2_rn(make_float2(e2s[0], e2s[1]), vv);
+      s.a = fmaf(e1s[0], s.a, ev.x);
+      s.b = fmaf(e1s[0], s.b, e2s[0]);
+      s.a = fmaf(e1s[1], s.a, ev.y);
+      s.b = fmaf(e1s[1], s.b, e2s[1]);
     }
   } else {
     int j = 0;
@@ -372,20 +396,27 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
   __shared__ float4 sfold[kFoldF][32];  // earlier segments' aggregates
   __shared__ float4 sin_[32];           // the state entering the segment
   __shared__ uint64_t bars[kSW];
-  __shared__ unsigned s_ticket;
+  __shared__ unsigned s_ticket[3];
 
   const int G = (C + 31) >> 5;
   const int64_t nbg = int64_t(B) * G;
   const int nch = (T + kTT - 1) / kTT;
   const int nseg = (nch + kSegC - 1) / kSegC;
   const BwdLayout lay = bwd_layout(ws, B, T, C);
-  if (threadIdx.x == 0) s_ticket = atomicAdd(lay.fticket, 1u);
+  if (threadIdx.x == 0) {  // ticket -> (segment, batch row, channel group), decoded once
+    const unsigned ticket = atomicAdd(lay.fticket, 1u);  // < 2^31 (host check)
+    const unsigned sg = ticket / unsigned(nbg);
+    const unsigned r = ticket - sg * unsigned(nbg);
+    const unsigned bb = r / unsigned(G);
+    s_ticket[0] = sg;
+    s_ticket[1] = bb;
+    s_ticket[2] = r - bb * unsigned(G);
+  }
   __syncthreads();
-  const int64_t ticket = s_ticket;
-  const int seg = int(ticket / nbg);
-  const int64_t bg = ticket - int64_t(seg) * nbg;
-  const int b = int(bg / G);
-  const int g = int(bg - int64_t(b) * G);
+  const int seg = int(s_ticket[0]);
+  const int b = int(s_ticket[1]);
+  const int g = int(s_ticket[2]);
+  const int64_t bg = int64_t(b) * G + g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = (g << 5) + lane;
   const bool valid = c < C;
@@ -432,7 +463,7 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
   }
 
   // ---- the chunks' aggregates from the empty state ----
-  if (ch0 < nch) mbar_wait(bar, 0, err);
+  if (ch0 < nch) mbar_wait_suspend(bar, 0, err);
   __syncwarp();
 #pragma unroll
   for (int q = 0; q < kCK; ++q) {
@@ -826,13 +857,136 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
   return A;
 }
 
+// chunk_forward in the single-exponential output form with the work off the serial chains
+// two tokens to an fp32x2 instruction. The chains stay scalar, token by token, in the same
+// operations as absorb_indep (so the state after the chunk is bit for bit the checkpoint
+// pass's): the scale (d, the takeover selects, the window rebase), a and b, and the
+// running product E of the map. Each token's a, b and E before it land in its half of a
+// register pair for the packed output, gate, factor and dr arithmetic, whose lanes round
+// as the scalar forms. The map's sums (lb, lg, lbd, lgd) are kept as even- and odd-token
+// partial sums, added at the end.
+template <bool GATE, bool DR, int RB>
+__device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanParams& cp, float* K,
+                                                      const float* V, float* R, float* DY,
+                                                      ChunkFactors& f) {
+  static_assert(kTT % RB == 0 && kTT % 2 == 0, "windows and pairs must tile the chunk");
+  const float2 l2e = make_float2(kLog2e, kLog2e);
+  const float2 w2 = make_float2(cp.w2, cp.w2);
+  const float2 H = make_float2(cp.H, cp.H);
+  float E = 1.f, a = s.a, b = s.b, Q = s.Q, pl = s.pl;
+  float2 lb = make_float2(0.f, 0.f), lg = lb, lbd = lb, lgd = lb;
+  f.tok = 0u;
+#pragma unroll
+  for (int t = 0; t < kTT; t += 2) {
+    const float2 kk = make_float2(K[t * 32], K[(t + 1) * 32]);
+    const float2 vv = make_float2(V[t * 32], V[(t + 1) * 32]);
+    const float2 gy = make_float2(DY[t * 32], DY[(t + 1) * 32]);
+    // tok_log2w of both tokens: the product rounded on its own, then the fma
+    const float2 m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
+                                __fmul2_rn(kk, l2e));
+    float2 sig = make_float2(1.f, 1.f);
+    if (GATE) {
+      const float2 x = __fmul2_rn(make_float2(R[t * 32], R[(t + 1) * 32]),
+                                  make_float2(-kLog2e, -kLog2e));
+      const float2 q = __fadd2_rn(make_float2(ex2(x.x), ex2(x.y)), make_float2(1.f, 1.f));
+      sig = make_float2(rcp(q.x), rcp(q.y));
+    }
+    // the scale chain, token t then t + 1 (as absorb_indep)
+    float ee[2], e1s[2], e2s[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float mh = h ? m.y : m.x;
+      const float d = (mh - Q) - pl;
+      ee[h] = ex2(-fabsf(d));
+      const bool cnd = d > 0.f;
+      e1s[h] = cnd ? ee[h] : 1.f;
+      e2s[h] = cnd ? 1.f : ee[h];
+      Q = cnd ? mh : Q;
+      pl = cnd ? 0.f : pl;
+      f.tok |= cnd ? (1u << (t + h)) : 0u;
+      if ((t + h + 1) % RB == 0) {
+        ChanState r;
+        r.Q = Q;
+        r.pl = pl;
+        wkv_rebase(r, float(RB) * cp.w2);
+        Q = r.Q;
+        pl = r.pl;
+      }
+    }
+    f.fe[t] = ee[0];
+    f.fe[t + 1] = ee[1];
+    const float2 e1 = make_float2(e1s[0], e1s[1]);
+    const float2 e2 = make_float2(e2s[0], e2s[1]);
+    // the a, b and E chains; each value before its token kept for the pair
+    const float2 ev = __fmul2_rn(e2, vv);
+    float2 ap, bp, Ep;
+    ap.x = a;
+    bp.x = b;
+    Ep.x = E;
+    a = fmaf(e1.x, a, ev.x);
+    b = fmaf(e1.x, b, e2.x);
+    E *= e1.x;
+    ap.y = a;
+    bp.y = b;
+    Ep.y = E;
+    a = fmaf(e1.y, a, ev.y);
+    b = fmaf(e1.y, b, e2.y);
+    E *= e1.y;
+    // output, factors, dr, and the map's sums
+    const float2 he = __fmul2_rn(H, e2);
+    const float2 num = __ffma2_rn(e1, ap, __fmul2_rn(he, vv));
+    const float2 den = __ffma2_rn(e1, bp, he);
+    const float2 rden = make_float2(rcp(den.x), rcp(den.y));
+    const float2 hh = __fmul2_rn(__fmul2_rn(gy, sig), rden);  // dy sigmoid(r) / den
+    const float2 wk = __fmul2_rn(num, rden);
+    const float2 inj = __fmul2_rn(hh, e1);
+    f.inj[t] = inj.x;
+    f.inj[t + 1] = inj.y;
+    K[t * 32] = wk.x;
+    K[(t + 1) * 32] = wk.y;
+    const float2 cur = __fmul2_rn(hh, he);
+    DY[t * 32] = cur.x;
+    DY[(t + 1) * 32] = cur.y;
+    if (DR) {
+      const float2 dr = __fmul2_rn(__fmul2_rn(__fmul2_rn(gy, wk), sig),
+                                   __ffma2_rn(sig, make_float2(-1.f, -1.f), make_float2(1.f, 1.f)));
+      R[t * 32] = dr.x;
+      R[(t + 1) * 32] = dr.y;
+    }
+    const float2 ej = __fmul2_rn(Ep, inj);
+    const float2 tt = make_float2(float(t), float(t + 1));
+    lbd = __ffma2_rn(ej, tt, lbd);
+    lgd = __ffma2_rn(__fmul2_rn(ej, wk), tt, lgd);
+    lb = __fadd2_rn(lb, ej);
+    lg = __ffma2_rn(ej, wk, lg);
+  }
+  s.a = a;
+  s.b = b;
+  s.Q = Q;
+  s.pl = pl;
+  RevAgg A;
+  A.E = E;
+  A.L = float(kTT);
+  A.lb = lb.x + lb.y;
+  A.lg = lg.x + lg.y;
+  A.lbd = lbd.x + lbd.y;
+  A.lgd = lgd.x + lgd.y;
+  return A;
+}
+
 template <bool GATE, bool DR, bool FASTOUT>
 __device__ __forceinline__ RevAgg chunk_forward_rb(ChanState& s, const ChanParams& cp, int rb,
                                                    float* K, const float* V, float* R, float* DY,
                                                    ChunkFactors& f) {
-  if (rb == 16) return chunk_forward<GATE, DR, FASTOUT, 16>(s, cp, K, V, R, DY, f);
-  if (rb == 4) return chunk_forward<GATE, DR, FASTOUT, 4>(s, cp, K, V, R, DY, f);
-  return chunk_forward<GATE, DR, FASTOUT, 1>(s, cp, K, V, R, DY, f);
+  if constexpr (FASTOUT) {
+    if (rb == 16) return chunk_forward_pairs<GATE, DR, 16>(s, cp, K, V, R, DY, f);
+    if (rb == 4) return chunk_forward_pairs<GATE, DR, 4>(s, cp, K, V, R, DY, f);
+    return chunk_forward_pairs<GATE, DR, 1>(s, cp, K, V, R, DY, f);
+  } else {
+    if (rb == 16) return chunk_forward<GATE, DR, false, 16>(s, cp, K, V, R, DY, f);
+    if (rb == 4) return chunk_forward<GATE, DR, false, 4>(s, cp, K, V, R, DY, f);
+    return chunk_forward<GATE, DR, false, 1>(s, cp, K, V, R, DY, f);
+  }
 }
 
 // Reverse over one chunk from the carry X after its last real token (position nvalid - 1;
@@ -863,6 +1017,57 @@ __device__ __forceinline__ float2 chunk_reverse(const ChunkFactors& f, RevCarry 
   return make_float2(-dw_acc, du_acc);
 }
 
+// chunk_reverse over a whole chunk with the work off the carry's chains two tokens (t and
+// t - 1) to an fp32x2 instruction. The chains stay scalar, token by token, and carry -gamma
+// and -gammad in place of gamma and gammad (negation is exact, so every value is the
+// scalar form's, with the subtractions dk and dw need turned into the fma's own add). The
+// carry before each token lands in its half of a register pair for dv, dk and the dw, du
+// terms; dw and du are kept as partial sums by token parity.
+__device__ __forceinline__ float2 chunk_reverse_pairs(const ChunkFactors& f, RevCarry X, float* K,
+                                                      float* V, const float* CUR) {
+  static_assert(kTT % 2 == 0, "pairs must tile the chunk");
+  float xb = X.b, ng = -X.g, xbd = X.bd, ngd = -X.gd;
+  float2 dw = make_float2(0.f, 0.f), du = dw;
+#pragma unroll
+  for (int t = kTT - 1; t > 0; t -= 2) {
+    const float2 vv = make_float2(V[t * 32], V[(t - 1) * 32]);
+    const float2 wk = make_float2(K[t * 32], K[(t - 1) * 32]);
+    const float2 cur = make_float2(CUR[t * 32], CUR[(t - 1) * 32]);
+    const float2 inj = make_float2(f.inj[t], f.inj[t - 1]);
+    const bool d0 = (f.tok >> t) & 1u, d1 = (f.tok >> (t - 1)) & 1u;
+    const float2 e1 = make_float2(d0 ? f.fe[t] : 1.f, d1 ? f.fe[t - 1] : 1.f);
+    const float2 e2 = make_float2(d0 ? 1.f : f.fe[t], d1 ? 1.f : f.fe[t - 1]);
+    const float2 iw = __fmul2_rn(inj, wk);
+    float2 pb, png, pbd, pngd;  // the carry before each token of the pair
+    pb.x = xb;
+    png.x = ng;
+    pbd.x = xbd;
+    pngd.x = ngd;
+    xbd = e1.x * (xbd + xb);
+    ngd = e1.x * (ngd + ng);
+    xb = fmaf(e1.x, xb, inj.x);
+    ng = fmaf(e1.x, ng, -iw.x);
+    pb.y = xb;
+    png.y = ng;
+    pbd.y = xbd;
+    pngd.y = ngd;
+    xbd = e1.y * (xbd + xb);
+    ngd = e1.y * (ngd + ng);
+    xb = fmaf(e1.y, xb, inj.y);
+    ng = fmaf(e1.y, ng, -iw.y);
+    const float2 vm = __ffma2_rn(wk, make_float2(-1.f, -1.f), vv);  // v - wkv
+    const float2 dv = __ffma2_rn(e2, pb, cur);
+    const float2 dk = __ffma2_rn(cur, vm, __fmul2_rn(e2, __ffma2_rn(vv, pb, png)));
+    dw = __ffma2_rn(e2, __ffma2_rn(vv, pbd, pngd), dw);
+    du = __ffma2_rn(cur, vm, du);
+    V[t * 32] = dv.x;
+    V[(t - 1) * 32] = dv.y;
+    K[t * 32] = dk.x;
+    K[(t - 1) * 32] = dk.y;
+  }
+  return make_float2(-(dw.x + dw.y), du.x + du.y);
+}
+
 // One CTA per (segment of kSW chunks, batch row, 32-channel group); warp i owns chunk
 // kSW seg + i. CTAs take segments in ticket order from the LAST segment backward, so every
 // segment a CTA waits for belongs to a CTA that started earlier: the waits always end.
@@ -891,7 +1096,7 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   __shared__ float4 sfold[2 * kFoldR + 1][32];  // later segments' maps and carry
   __shared__ float4 sxe[32];                    // the carry at the segment's end
   __shared__ uint64_t bars[kSW];
-  __shared__ unsigned s_tk;
+  __shared__ unsigned s_tk[3];
   // The chunks' partial sums (-dw, du), in sfold's space (used at other times).
   static_assert(2 * kFoldR + 1 >= kSW / 2, "spart must fit in sfold");
   auto spart = reinterpret_cast<float2(*)[32]>(&sfold[0][0]);
@@ -902,14 +1107,20 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   const int nseg = (nch + kSW - 1) / kSW;
   const BwdLayout lay = bwd_layout(ws, B, T, C);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) s_tk = atomicAdd(lay.rticket, 1u);
+  if (threadIdx.x == 0) {  // ticket -> (segments from the end, batch row, channel group)
+    const unsigned tk = atomicAdd(lay.rticket, 1u);  // < 2^31 (host check)
+    const unsigned bk = tk / unsigned(nbg);
+    const unsigned r = tk - bk * unsigned(nbg);
+    const unsigned bb = r / unsigned(G);
+    s_tk[0] = bk;
+    s_tk[1] = bb;
+    s_tk[2] = r - bb * unsigned(G);
+  }
   __syncthreads();
-  const unsigned tk = s_tk;
-  const int back = int(tk / nbg);  // segments from the end
-  const int seg = nseg - 1 - back;
-  const int64_t bg = int64_t(tk) - int64_t(back) * nbg;
-  const int b = int(bg / G);
-  const int g = int(bg - int64_t(b) * G);
+  const int seg = nseg - 1 - int(s_tk[0]);
+  const int b = int(s_tk[1]);
+  const int g = int(s_tk[2]);
+  const int64_t bg = int64_t(b) * G + g;
   const int c = (g << 5) + lane;
   const bool valid = c < C;
   const int ch = seg * kSW + warp;
@@ -976,7 +1187,7 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   s.Q = ck.z;
   s.pl = ck.w;
   if (live) {
-    mbar_wait(bar, 0, err);
+    mbar_wait_suspend(bar, 0, err);
     __syncwarp();
     // Past the last token (zero-filled tiles): a weight of 2^{-huge} makes the positions
     // inert (e1 = 1, e2 = 0: the state and the reverse sums pass through unchanged).
@@ -1068,7 +1279,7 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   float2 part = make_float2(0.f, 0.f);
   if (live) {
     const RevCarry Xc{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme};
-    part = nvalid == kTT ? chunk_reverse<false>(f, Xc, K, V, DY, kTT)
+    part = nvalid == kTT ? chunk_reverse_pairs(f, Xc, K, V, DY)
                          : chunk_reverse<true>(f, Xc, K, V, DY, nvalid);
     fence_proxy_async_smem();
     __syncwarp();

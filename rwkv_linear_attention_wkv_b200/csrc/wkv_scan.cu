@@ -97,20 +97,27 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   float4* sin = sagg + kW * 32;                                            // [32]
   float4* sfold = sin + 32;                                                // [kFold][32]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sfold + kFold * 32);         // [W]
-  __shared__ unsigned s_ticket;
+  __shared__ unsigned s_ticket[3];
 
   const int G = (C + 31) >> 5;
   const int64_t nbg = int64_t(B) * G;
   const ScanLayout lay = scan_layout(scratch, nbg * nseg);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) s_ticket = atomicAdd(lay.ticket, 1u);
+  if (threadIdx.x == 0) {  // ticket -> (segment, batch row, channel group), decoded once
+    const unsigned ticket = atomicAdd(lay.ticket, 1u);  // < 2^31 (host check)
+    const unsigned sg = ticket / unsigned(nbg);
+    const unsigned r = ticket - sg * unsigned(nbg);
+    const unsigned bb = r / unsigned(G);
+    s_ticket[0] = sg;
+    s_ticket[1] = bb;
+    s_ticket[2] = r - bb * unsigned(G);
+  }
   __syncthreads();
-  const int64_t ticket = s_ticket;
-  const int seg = int(ticket / nbg);
-  const int64_t bg = ticket - int64_t(seg) * nbg;
-  const int b = int(bg / G);
-  const int g = int(bg - int64_t(b) * G);
+  const int seg = int(s_ticket[0]);
+  const int b = int(s_ticket[1]);
+  const int g = int(s_ticket[2]);
+  const int64_t bg = int64_t(b) * G + g;
   const int c = (g << 5) + lane;
   const bool valid = c < C;
   const int64_t item0 = bg * nseg;
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(kW * 32) wkv_fwd_chunked_kernel(
   }
 
   // ---- 1. sub-chunk aggregate from the empty state ----
-  if (n > 0) mbar_wait(bar, 0, err);
+  if (n > 0) mbar_wait_suspend(bar, 0, err);
   __syncwarp();
   ChanState s = empty_state();
   if (n == kLS) {
