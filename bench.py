@@ -286,27 +286,60 @@ def run_ours(args, rank, world, local_rank):
         [starts[0].elapsed_time(ends[-1]), statistics.mean(per_launch)], dist, dev)
     value = aggregate_rate(world, ELEMS, args.steps, elapsed_ms)
 
-    # End to end through the public API: pinned host k, v, r -> device, forward, y -> host.
+    # End to end through the public API: pinned host k, v, r -> device, forward, y -> host,
+    # every step. Steps are pipelined over two device buffer sets and three streams (copy
+    # in, compute, copy out): PCIe is full duplex, so one step's inputs go up while the
+    # previous step's output comes down. A set's inputs are overwritten only after the
+    # kernel that read them has finished, and its y only after it has been copied out.
     e2e_steps = max(3, min(args.steps, 20))
     hk, hv, hr = (to_bf16(x.bits[n], pin=True) for n in "kvr")
     hy = torch.empty(hk.shape, dtype=torch.bfloat16).pin_memory()
-    dk, dv, dr, dy_ = (torch.empty_like(k) for _ in range(4))
+    bufs = [tuple(torch.empty_like(k) for _ in range(4)) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    consumed = [None, None]  # set j's inputs read by its last kernel
+    drained = [None, None]   # set j's y copied to the host
 
-    def e2e_step():
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dr.copy_(hr, non_blocking=True)
-        W.wkv_forward_bf16(w, u, dk, dv, dr, y=dy_)
-        hy.copy_(dy_, non_blocking=True)
+    def e2e_step(i):
+        j = i % 2
+        dk, dv, dr, dy_ = bufs[j]
+        if consumed[j] is not None:
+            s_in.wait_event(consumed[j])
+        with torch.cuda.stream(s_in):
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dr.copy_(hr, non_blocking=True)
+        loaded = torch.cuda.Event()
+        loaded.record(s_in)
+        stream.wait_event(loaded)
+        if drained[j] is not None:
+            stream.wait_event(drained[j])
+        W.wkv_forward_bf16(w, u, dk, dv, dr, y=dy_, stream=stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        consumed[j] = done
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            hy.copy_(dy_, non_blocking=True)
+        out = torch.cuda.Event()
+        out.record(s_out)
+        drained[j] = out
 
-    for _ in range(2):
-        e2e_step()
+    def e2e_drain():
+        for ev in drained:
+            if ev is not None:
+                stream.wait_event(ev)
+
+    for i in range(2):
+        e2e_step(i)
+    e2e_drain()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e2e_drain()
     e1.record(stream)
     barrier()
     (e2e_ms,) = max_over_ranks([e0.elapsed_time(e1)], dist, dev)
