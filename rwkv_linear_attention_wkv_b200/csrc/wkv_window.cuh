@@ -12,23 +12,11 @@ namespace wkv {
 // has (a running max for the scale, one fma per token for a and b): every load of the
 // window first, then the log-weights and their running max, then the per-token
 // arithmetic, then every store. (Token by token, each token's loads would wait for the
-// previous token's store, which the compiler must assume may alias them.)
-//
-// In the single-exponential output form, windows of two or more tokens go through
-// window_fast_pairs: the same operations with the ones that do not lie on the recurrence's
-// serial chains packed two tokens to an fp32x2 instruction.
-template <typename Tin, bool GATE, int RB, int RS>
-__device__ __forceinline__ void window_fast_pairs(ChanState& s, const ChanParams& cp,
-                                                  const Tin* K, const Tin* V, const Tin* R,
-                                                  Tin* Y);
-
+// previous token's store, which the compiler must assume may alias them.) Every token in
+// scalar instructions; see window_smem for the form that is used.
 template <typename Tin, bool GATE, bool FASTOUT, int RB, int RS>
-__device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, const Tin* K,
-                                            const Tin* V, const Tin* R, Tin* Y) {
-  if constexpr (FASTOUT && RB >= 2) {
-    window_fast_pairs<Tin, GATE, RB, RS>(s, cp, K, V, R, Y);
-    return;
-  }
+__device__ __forceinline__ void window_scalar(ChanState& s, const ChanParams& cp, const Tin* K,
+                                              const Tin* V, const Tin* R, Tin* Y) {
   float kk[RB], vv[RB], m[RB], d[RB], den[RB], num[RB];
   float rr[GATE ? RB : 1];
 #pragma unroll
@@ -174,6 +162,19 @@ __device__ __forceinline__ void window_fast_pairs(ChanState& s, const ChanParams
     Y[(2 * i + 1) * RS] = Elem<Tin>::from_f(y.y);
   }
   wkv_rebase(s, float(RB) * cp.w2);
+}
+
+// One full window of RB tokens: in the single-exponential output form, windows of two or
+// more tokens go through window_fast_pairs (the operations off the recurrence's serial
+// chains packed two tokens to an fp32x2 instruction, same results); otherwise
+// window_scalar.
+template <typename Tin, bool GATE, bool FASTOUT, int RB, int RS>
+__device__ __forceinline__ void window_smem(ChanState& s, const ChanParams& cp, const Tin* K,
+                                            const Tin* V, const Tin* R, Tin* Y) {
+  if constexpr (FASTOUT && RB >= 2)
+    window_fast_pairs<Tin, GATE, RB, RS>(s, cp, K, V, R, Y);
+  else
+    window_scalar<Tin, GATE, FASTOUT, RB, RS>(s, cp, K, V, R, Y);
 }
 
 // Process n tokens of a tile in shared memory (row stride RS, this thread's column).
