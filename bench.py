@@ -457,6 +457,31 @@ def run_workload(args):
                         args.steps, args.warmup, stream)
         line("train_169m", "backward_state fp32 16x1024x768 (with initial state and final-state "
              "gradients)", ms, n, 28 * n + 36 * x.B * x.C)
+        # The checkpointed pair: the forward also writes the backward's chunk checkpoints
+        # (one float4 per channel per 16 tokens: 1 byte per element), the backward reads
+        # them instead of forming them in a pass of its own.
+        ms_f = _time_loop(lambda: W.wkv_forward_checkpointed(w, u, k, v, r, y=y, workspace=ws),
+                          args.steps, args.warmup, stream)
+        line("train_169m", "forward_checkpointed fp32 16x1024x768 (y and the backward's "
+             "checkpoints)", ms_f, n, 17 * n)
+        ms_b = _time_loop(lambda: W.wkv_backward_checkpointed(w, u, k, v, r, dy, ws, out=out),
+                          args.steps, args.warmup, stream)
+        line("train_169m", "backward_checkpointed fp32 16x1024x768 (dk, dv, dr, dw, du; "
+             "checkpoints read)", ms_b, n, 29 * n)
+
+        def step_plain():
+            W.wkv_forward(w, u, k, v, r, y=y)
+            W.wkv_backward(w, u, k, v, r, dy, workspace=ws, out=out)
+
+        def step_ckpt():
+            W.wkv_forward_checkpointed(w, u, k, v, r, y=y, workspace=ws)
+            W.wkv_backward_checkpointed(w, u, k, v, r, dy, ws, out=out)
+
+        ms_p = _time_loop(step_plain, args.steps, args.warmup, stream)
+        ms_c = _time_loop(step_ckpt, args.steps, args.warmup, stream)
+        line("train_169m", "training step: wkv_forward + wkv_backward", ms_p, n, 16 * n + 28 * n)
+        line("train_169m", "training step: wkv_forward_checkpointed + wkv_backward_checkpointed",
+             ms_c, n, 17 * n + 29 * n)
     elif args.workload == "long_ctx":
         x = wkv_inputs.long_context(seed=0, T=args.seq or 32768)
         w, u, k, v, r = (d(a) for a in (x.w, x.u, x.k, x.v, x.r))

@@ -205,6 +205,40 @@ WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, 
                                cudaStream_t stream);
 
 /*
+ * Training step with the checkpoints made by the forward. The backward (wkv_backward,
+ * wkv_backward_state) spends about a quarter of its time on a pass over k and v that forms
+ * the state entering every chunk of 16 tokens; in training the forward has just walked the
+ * same tokens, so wkv_forward_checkpointed writes those states (1 byte per element) into the
+ * backward's workspace as it goes, and wkv_backward_checkpointed, given that workspace,
+ * skips the pass.
+ *
+ * wkv_forward_checkpointed: y as wkv_forward_state (initial state a0, b0, p0 or all NULL;
+ *   no final state), fp32, and the checkpoints into `workspace` (device, 256-byte aligned,
+ *   at least wkv_backward_workspace_bytes(B, T, C) bytes, owned by the caller and kept
+ *   unchanged until the backward). Its per-token scale arithmetic is the backward's, so y
+ *   rounds differently from wkv_forward's (within the same tolerance of the exact result).
+ *   Needs the shapes of the streaming kernel: C a multiple of 4 and k, v, r, y 16-byte
+ *   aligned, else WKV_ERR_UNSUPPORTED. Errors as wkv_forward_state; a missing or short
+ *   workspace is WKV_ERR_INVALID_ARG. T == 0: nothing is written.
+ * wkv_backward_checkpointed: arguments and results as wkv_backward_state; `workspace` must
+ *   be the one the forward filled, with the same B, T, C, w, u, k, v and initial state
+ *   (nothing checks this: other inputs give wrong gradients). Needs C a multiple of 4 and
+ *   k, v, r, dy, dk, dv, dr 16-byte aligned, else WKV_ERR_UNSUPPORTED. The checkpoints are
+ *   read, not changed: one forward can serve several backward calls. Deterministic.
+ */
+WKV_API int wkv_forward_checkpointed(int64_t B, int64_t T, int64_t C, const float* w,
+                                     const float* u, const float* k, const float* v,
+                                     const float* r, float* y, const float* a0, const float* b0,
+                                     const float* p0, void* workspace, size_t workspace_bytes,
+                                     cudaStream_t stream);
+WKV_API int wkv_backward_checkpointed(
+    int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+    const float* v, const float* r, const float* dy, const float* a0, const float* b0,
+    const float* p0, const float* ga1, const float* gb1, const float* p1, float* dk, float* dv,
+    float* dw, float* du, float* dr, float* da0, float* db0, float* dp0, void* workspace,
+    size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * RWKV-7 recurrence per head, fp32 (research report "RWKV模型深度研究报告（截至2026年初）",
  * section 1.3.3 "RWKV-7 (Goose)": the generalised-delta-rule state update
  *   S_t = S_{t-1} (diag(w_t) + a_t^T b_t) + v_t^T k_t

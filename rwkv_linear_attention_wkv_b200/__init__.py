@@ -13,6 +13,7 @@ import os
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
            "wkv_backward", "wkv_backward_state", "wkv_backward_workspace_bytes",
+           "wkv_forward_checkpointed", "wkv_backward_checkpointed",
            "wkv7_forward", "wkv_stream_status", "wkv_status_string", "WkvError", "lib",
            "LIB_PATH"]
 
@@ -41,6 +42,9 @@ _SIGS = {
                                    ctypes.c_int),
     "wkv_backward_state": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int),
     "wkv7_forward": ([_I, _I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
+    "wkv_forward_checkpointed": ([_I, _I, _I] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int),
+    "wkv_backward_checkpointed": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
+                                  ctypes.c_int),
     "wkv_testing_backward_state_plain": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
                                          ctypes.c_int),
     "wkv_testing_lookback_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
@@ -285,6 +289,55 @@ def wkv_backward_state(w, u, k, v, r, dy, state=None, grad_state=None, want_dr=T
           _ptr(out["da0"]), _ptr(out["db0"]), _ptr(out["dp0"]),
           _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     return out
+
+
+def wkv_forward_checkpointed(w, u, k, v, r=None, state=None, y=None, workspace=None,
+                             stream=None):
+    """fp32 forward of a training step that also writes the backward's checkpoints.
+
+    y as wkv_forward_state(w, u, k, v, r, state) (no final state); the checkpoints go into
+    `workspace` (uint8 CUDA tensor of at least wkv_backward_workspace_bytes(B, T, C) bytes,
+    allocated when not given). Returns (y, workspace); hand the workspace, unchanged, to
+    wkv_backward_checkpointed with the same w, u, k, v and state.
+    """
+    torch = _torch()
+    f32 = torch.float32
+    if k.dim() != 3:
+        raise ValueError("k must be (B, T, C)")
+    B, T, C = k.shape
+    _need(k, "k", f32)
+    _need(v, "v", f32, (B, T, C))
+    if r is not None:
+        _need(r, "r", f32, (B, T, C))
+    _need(w, "w", f32, (C,))
+    _need(u, "u", f32, (C,))
+    st = tuple(state) if state is not None else (None, None, None)
+    for n, t in zip(("a0", "b0", "p0"), st):
+        if t is not None:
+            _need(t, n, f32, (B, C))
+    if y is None:
+        y = torch.empty((B, T, C), dtype=f32, device=k.device)
+    _need(y, "y", f32, (B, T, C))
+    nbytes = wkv_backward_workspace_bytes(B, T, C)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=k.device)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA tensor of at least {nbytes} bytes")
+    _call("wkv_forward_checkpointed", B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+          _ptr(y), *(_ptr(t) for t in st), _ptr(workspace),
+          workspace.numel() * workspace.element_size(), _stream(stream))
+    return y, workspace
+
+
+def wkv_backward_checkpointed(w, u, k, v, r, dy, workspace, state=None, grad_state=None,
+                              want_dr=True, out=None, stream=None):
+    """wkv_backward_state, using the checkpoints wkv_forward_checkpointed left in
+    `workspace` (same w, u, k, v and state) instead of forming them again."""
+    if workspace is None:
+        raise ValueError("workspace: the one wkv_forward_checkpointed filled")
+    return wkv_backward_state(w, u, k, v, r, dy, state=state, grad_state=grad_state,
+                              want_dr=want_dr, workspace=workspace, out=out, stream=stream,
+                              _entry="wkv_backward_checkpointed")
 
 
 def wkv7_forward(r, w, k, v, a, b, state=None, y=None, state_out=None, want_state=True,

@@ -146,7 +146,7 @@ static int backward_impl(int64_t B, int64_t T, int64_t C, const float* w, const 
                          const float* k, const float* v, const float* r, const float* dy,
                          float* dk, float* dv, float* dw, float* du, float* dr, void* workspace,
                          size_t workspace_bytes, bool force_plain, cudaStream_t stream,
-                         const StateArgs& st = StateArgs()) {
+                         const StateArgs& st = StateArgs(), bool have_ckpt = false) {
   if (B < 0 || T < 0 || C < 0) return WKV_ERR_INVALID_ARG;
   if (!all_or_none(st.a0, st.b0, st.p0) || !all_or_none(st.ga1, st.gb1, st.p1) ||
       !all_or_none(st.da0, st.db0, st.dp0))
@@ -185,7 +185,29 @@ static int backward_impl(int64_t B, int64_t T, int64_t C, const float* w, const 
   a.a0 = st.a0; a.b0 = st.b0; a.p0 = st.p0;
   a.ga1 = st.ga1; a.gb1 = st.gb1; a.p1 = st.p1;
   a.da0 = st.da0; a.db0 = st.db0; a.dp0 = st.dp0;
+  a.have_ckpt = have_ckpt ? 1 : 0;
   return launch_backward(a, force_plain, stream);
+}
+
+// wkv_forward_checkpointed: the forward of wkv_forward_state (without the final state) that
+// also writes the backward's checkpoints into `workspace`.
+static int forward_ckpt_impl(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
+                             const float* k, const float* v, const float* r, float* y,
+                             const float* a0, const float* b0, const float* p0, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_fwd(B, T, C, w, u, k, v, r, y, 4);
+  if (rc != WKV_OK) return rc;
+  if (!state_triplet_ok(a0, b0, p0)) return WKV_ERR_INVALID_ARG;
+  if (!aligned(a0, 4) || !aligned(b0, 4) || !aligned(p0, 4)) return WKV_ERR_ALIGNMENT;
+  if (B == 0 || C == 0 || T == 0) return WKV_OK;
+  if (B * ((C + 31) / 32) >= (int64_t(1) << 31)) return WKV_ERR_UNSUPPORTED;
+  if (workspace == nullptr || !aligned(workspace, 256) ||
+      workspace_bytes < backward_workspace_bytes(B, T, C))
+    return WKV_ERR_INVALID_ARG;
+  unsigned* err = error_word();
+  if (err == nullptr) return WKV_ERR_CUDA;
+  FwdArgs a{B, T, C, w, u, k, v, r, y, a0, b0, p0, nullptr, nullptr, nullptr, err};
+  return launch_fwd_ckpt(a, workspace, stream);
 }
 
 }  // namespace wkv
@@ -270,6 +292,29 @@ WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, 
   st.da0 = da0; st.db0 = db0; st.dp0 = dp0;
   return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
                        workspace_bytes, false, stream, st);
+}
+
+WKV_API int wkv_forward_checkpointed(int64_t B, int64_t T, int64_t C, const float* w,
+                                     const float* u, const float* k, const float* v,
+                                     const float* r, float* y, const float* a0, const float* b0,
+                                     const float* p0, void* workspace, size_t workspace_bytes,
+                                     cudaStream_t stream) {
+  return forward_ckpt_impl(B, T, C, w, u, k, v, r, y, a0, b0, p0, workspace, workspace_bytes,
+                           stream);
+}
+
+WKV_API int wkv_backward_checkpointed(
+    int64_t B, int64_t T, int64_t C, const float* w, const float* u, const float* k,
+    const float* v, const float* r, const float* dy, const float* a0, const float* b0,
+    const float* p0, const float* ga1, const float* gb1, const float* p1, float* dk, float* dv,
+    float* dw, float* du, float* dr, float* da0, float* db0, float* dp0, void* workspace,
+    size_t workspace_bytes, cudaStream_t stream) {
+  StateArgs st;
+  st.a0 = a0; st.b0 = b0; st.p0 = p0;
+  st.ga1 = ga1; st.gb1 = gb1; st.p1 = p1;
+  st.da0 = da0; st.db0 = db0; st.dp0 = dp0;
+  return backward_impl(B, T, C, w, u, k, v, r, dy, dk, dv, dw, du, dr, workspace,
+                       workspace_bytes, false, stream, st, /*have_ckpt=*/true);
 }
 
 WKV_API int wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float* r,

@@ -42,6 +42,7 @@
 
 #include "wkv_internal.h"
 #include "wkv_async.cuh"
+#include "wkv_indep.cuh"
 #include "wkv_step.cuh"
 
 namespace wkv {
@@ -296,33 +297,13 @@ __global__ void __launch_bounds__(32, 8) wkv_bwd_ckpt_kernel(const __grid_consta
   if (valid) lay.ckend[int64_t(b) * C + c] = make_float4(s.a, s.b, s.Q, s.pl);
 }
 
-// Token weights for the time-parallel checkpoints and the recomputation that starts from
-// them. The checkpoint after a chunk is its entering state combined with the chunk's own
-// aggregate (from the empty state), while the reverse pass recomputes the same chunk from the
-// entering state; the two must weigh every token identically, or a dominant token (a
-// spike in k) would carry two different roundings of its weight into the two sides and
-// the reverse sums would be inconsistent at the level of ulp(k log2 e). So the token's
-// log2-weight in the window, m = k log2(e) + j w2, is rounded independently of the state,
-// and the state's low part enters only the comparison d = (m - Q) - pl; a token that
-// takes over the scale sets it to (m, 0).
-// The product is rounded on its own (__fmul_rn): with fj a compile-time 1 the compiler
-// could otherwise fuse it into the fma, and the two kernels would round differently.
-__device__ __forceinline__ float tok_log2w(float fj, float w2, float k) {
-  return fmaf(fj, w2, __fmul_rn(k, kLog2e));
-}
-
+// Token weights and the scale step of the time-parallel checkpoints and of the
+// recomputation that starts from them: wkv_indep.cuh.
 __device__ __forceinline__ void absorb_indep(ChanState& s, const ChanParams& cp, float fj, float k,
                                              float v) {
-  const float m = tok_log2w(fj, cp.w2, k);
-  const float d = (m - s.Q) - s.pl;
-  const float e = ex2(-fabsf(d));
-  const bool c = d > 0.f;
-  const float e1 = c ? e : 1.f;
-  const float e2 = c ? 1.f : e;
-  s.Q = c ? m : s.Q;
-  s.pl = c ? 0.f : s.pl;
-  s.a = fmaf(e1, s.a, e2 * v);
-  s.b = fmaf(e1, s.b, e2);
+  const ScaleStep st = indep_step(tok_log2w(fj, cp.w2, k), s.Q, s.pl);
+  s.a = fmaf(st.e1, s.a, st.e2 * v);
+  s.b = fmaf(st.e1, s.b, st.e2);
 }
 
 // Time-parallel form (TMA shapes). One CTA per (checkpoint segment of kSW x kCK chunks,
@@ -345,25 +326,18 @@ __device__ __forceinline__ Agg chunk_aggregate(const float* K, const float* V, i
   if (n == kTT) {
     // absorb_indep token by token, with the log-weights and the products e2 v two tokens
     // to an fp32x2 instruction (each lane rounded as the scalar form)
-    const float2 l2e = make_float2(kLog2e, kLog2e);
-    const float2 w2 = make_float2(cp.w2, cp.w2);
 #pragma unroll
     for (int t = 0; t < kTT; t += 2) {
       const float2 kk = make_float2(K[t * 32], K[(t + 1) * 32]);
       const float2 vv = make_float2(V[t * 32], V[(t + 1) * 32]);
-      const float2 m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
-                                  __fmul2_rn(kk, l2e));
+      const float2 m =
+          tok_log2w2(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), cp.w2, kk);
       float e1s[2], e2s[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const float mh = h ? m.y : m.x;
-        const float d = (mh - s.Q) - s.pl;
-        const float e = ex2(-fabsf(d));
-        const bool c = d > 0.f;
-        e1s[h] = c ? e : 1.f;
-        e2s[h] = c ? 1.f : e;
-        s.Q = c ? mh : s.Q;
-        s.pl = c ? 0.f : s.pl;
+        const ScaleStep st = indep_step(h ? m.y : m.x, s.Q, s.pl);
+        e1s[h] = st.e1;
+        e2s[h] = st.e2;
         if ((t + h + 1) % RB == 0) wkv_rebase(s, float(RB) * cp.w2);
       }
       const float2 ev = __fmul2_rn(make_float2(e2s[0], e2s[1]), vv);
@@ -793,7 +767,8 @@ struct ChunkFactors {
 // Forward recomputation of one chunk of kTT tokens from its entering state s (left holding
 // the state after the chunk): fills the per-token factors (wkv into K, cur into DY), writes
 // dr in place of r (DR), and returns the chunk's reverse map (its sums from a zero carry,
-// composed token by token in time order).
+// composed token by token in time order). Token by token, in either output form; the
+// single-exponential form goes through chunk_forward_pairs below.
 template <bool GATE, bool DR, bool FASTOUT, int RB>
 __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& cp, float* K,
                                                 const float* V, float* R, float* DY,
@@ -804,7 +779,7 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
 #pragma unroll
   for (int t = 0; t < kTT; ++t) {
     const float kk = K[t * 32], vv = V[t * 32], gy = DY[t * 32];
-    const float m = tok_log2w(float(t % RB + 1), cp.w2, kk);  // as absorb_indep
+    const float m = tok_log2w(float(t % RB + 1), cp.w2, kk);  // as indep_step
     const float d = (m - s.Q) - s.pl;
     const float e = ex2(-fabsf(d));
     const bool cnd = d > 0.f;
@@ -904,14 +879,7 @@ __device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanPa
       Q = cnd ? mh : Q;
       pl = cnd ? 0.f : pl;
       f.tok |= cnd ? (1u << (t + h)) : 0u;
-      if ((t + h + 1) % RB == 0) {
-        ChanState r;
-        r.Q = Q;
-        r.pl = pl;
-        wkv_rebase(r, float(RB) * cp.w2);
-        Q = r.Q;
-        pl = r.pl;
-      }
+      if ((t + h + 1) % RB == 0) indep_rebase(Q, pl, float(RB) * cp.w2);
     }
     f.fe[t] = ee[0];
     f.fe[t + 1] = ee[1];
@@ -1395,11 +1363,13 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     if (nitems >= (int64_t(1) << 31)) return WKV_ERR_UNSUPPORTED;
     if (cudaMemsetAsync(a.ws, 0, bwd_flag_bytes(a.B, a.T, a.C), stream) != cudaSuccess)
       return WKV_ERR_CUDA;
-    const int64_t nch = (a.T + kTT - 1) / kTT;
-    const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
-    wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
-        ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
-    if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
+    if (!a.have_ckpt) {
+      const int64_t nch = (a.T + kTT - 1) / kTT;
+      const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
+      wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
+          ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
+      if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
+    }
     if (a.r)
       rc = a.dr ? launch_seg<true, true>(a, in, out, nitems, stream)
                 : launch_seg<true, false>(a, in, out, nitems, stream);
@@ -1426,6 +1396,13 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
 
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C) { return bwd_bytes(B, T, C); }
 
+void backward_checkpoint_ptrs(void* ws, int64_t B, int64_t T, int64_t C, float4** ckpt,
+                              float4** ckend) {
+  const BwdLayout lay = bwd_layout(ws, B, T, C);
+  *ckpt = lay.ckpt;
+  *ckend = lay.ckend;
+}
+
 namespace {
 // No tokens: the final state is the initial one, so dL/dA0 = dL/dA_T = ga1 e^{-p1} and
 // da0 = e^{p0} dL/dA0 (the same for b); dp0 = a0 da0 + b0 db0.
@@ -1451,12 +1428,17 @@ int launch_backward_no_tokens(const BwdArgs& a, cudaStream_t stream) {
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
-int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream) {
+bool backward_time_parallel_ok(const BwdArgs& a) {
   auto al16 = [](const void* p) {
     return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0;
   };
-  const bool tma = !force_plain && a.C % 4 == 0 && al16(a.k) && al16(a.v) && al16(a.r) &&
-                   al16(a.dy) && al16(a.dk) && al16(a.dv) && al16(a.dr);
+  return a.C % 4 == 0 && al16(a.k) && al16(a.v) && al16(a.r) && al16(a.dy) && al16(a.dk) &&
+         al16(a.dv) && al16(a.dr);
+}
+
+int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream) {
+  const bool tma = !force_plain && backward_time_parallel_ok(a);
+  if (a.have_ckpt && !tma) return WKV_ERR_UNSUPPORTED;
   return tma ? launch_all<true>(a, stream) : launch_all<false>(a, stream);
 }
 

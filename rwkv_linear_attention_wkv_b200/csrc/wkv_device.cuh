@@ -95,17 +95,6 @@ __device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-// Acquire pattern completing a relaxed read of a flag: later reads see what the publisher
-// wrote before its release.
-__device__ __forceinline__ void fence_acquire() {
-  asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
-
 // Publishes *flag = v after this warp's earlier global writes; every lane calls it. The
 // warp barrier orders each lane's writes before lane 0's release store, and release is
 // cumulative, so a thread that acquires the flag sees all of them.

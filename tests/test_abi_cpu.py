@@ -116,3 +116,25 @@ def test_backward_state_argument_checks(W):
     assert call(2, full, full, [ok, ok, P(4098)]) == 2          # dp0 not 4-byte aligned
     assert call(-2, full, full, full) == 1
     assert call(0, full, full, full) == 0                       # no batch rows: nothing
+
+
+def test_checkpointed_pair_argument_checks(W):
+    # Refusals that happen before anything is enqueued (no GPU needed).
+    ok = P(4096)
+    need = W.wkv_backward_workspace_bytes(2, 64, 32)
+    fc = W.lib.wkv_forward_checkpointed
+    none3 = [None] * 3
+    assert fc(2, 64, 32, ok, ok, ok, ok, ok, ok, *none3, ok, need - 1, None) == 1  # short
+    assert fc(2, 64, 32, ok, ok, ok, ok, ok, ok, *none3, None, need, None) == 1    # no ws
+    assert fc(2, 64, 32, ok, ok, ok, ok, ok, ok, *none3, P(4352 + 16), need, None) == 1
+    assert fc(2, 64, 32, ok, ok, ok, ok, ok, ok, ok, None, ok, ok, need, None) == 1  # a0 triple
+    assert fc(2, 64, 32, ok, ok, ok, ok, ok, P(4098), *none3, ok, need, None) == 2   # y align
+    assert fc(-1, 64, 32, ok, ok, ok, ok, ok, ok, *none3, ok, need, None) == 1
+    assert fc(2, 0, 32, ok, ok, ok, ok, ok, ok, *none3, None, 0, None) == 0         # no tokens
+    bc = W.lib.wkv_backward_checkpointed
+    base = [ok] * 6
+    outs = [ok] * 5
+    assert bc(2, 64, 32, *base, *none3, *none3, *outs, *none3, ok, need - 1, None) == 1
+    assert bc(2, 64, 32, *base, [ok, None, ok][0], None, ok, *none3, *outs, *none3, ok, need,
+              None) == 1
+    assert bc(0, 64, 32, *base, *none3, *none3, *outs, *none3, ok, need, None) == 0
