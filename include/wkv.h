@@ -215,8 +215,9 @@ WKV_API int wkv_backward_state(int64_t B, int64_t T, int64_t C, const float* w, 
  * wkv_forward_checkpointed: y as wkv_forward_state (initial state a0, b0, p0 or all NULL;
  *   no final state), fp32, and the checkpoints into `workspace` (device, 256-byte aligned,
  *   at least wkv_backward_workspace_bytes(B, T, C) bytes, owned by the caller and kept
- *   unchanged until the backward). Its per-token scale arithmetic is the backward's, so y
- *   rounds differently from wkv_forward's (within the same tolerance of the exact result).
+ *   unchanged until the backward). y is bit for bit what wkv_forward's streaming kernel
+ *   computes (wkv_forward takes a chunked form instead below 8192 channels B*C, which
+ *   rounds differently); the backward then recomputes in that kernel's arithmetic.
  *   Needs the shapes of the streaming kernel: C a multiple of 4 and k, v, r, y 16-byte
  *   aligned, else WKV_ERR_UNSUPPORTED. Errors as wkv_forward_state; a missing or short
  *   workspace is WKV_ERR_INVALID_ARG. T == 0: nothing is written.

@@ -769,7 +769,7 @@ struct ChunkFactors {
 // dr in place of r (DR), and returns the chunk's reverse map (its sums from a zero carry,
 // composed token by token in time order). Token by token, in either output form; the
 // single-exponential form goes through chunk_forward_pairs below.
-template <bool GATE, bool DR, bool FASTOUT, int RB>
+template <bool GATE, bool DR, bool FASTOUT, int RB, bool FWD>
 __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& cp, float* K,
                                                 const float* V, float* R, float* DY,
                                                 ChunkFactors& f) {
@@ -779,14 +779,24 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
 #pragma unroll
   for (int t = 0; t < kTT; ++t) {
     const float kk = K[t * 32], vv = V[t * 32], gy = DY[t * 32];
-    const float m = tok_log2w(float(t % RB + 1), cp.w2, kk);  // as indep_step
-    const float d = (m - s.Q) - s.pl;
+    float m, d;
+    if (FWD) {  // the streaming forward's scale: m against the window start, running maximum
+      m = fmaf(float(t % RB + 1), cp.w2, fmaf(kk, kLog2e, -s.pl));
+      d = m - s.Q;
+    } else {  // as indep_step
+      m = tok_log2w(float(t % RB + 1), cp.w2, kk);
+      d = (m - s.Q) - s.pl;
+    }
     const float e = ex2(-fabsf(d));
     const bool cnd = d > 0.f;
     const float e1 = cnd ? e : 1.f;
     const float e2 = cnd ? 1.f : e;
-    s.Q = cnd ? m : s.Q;
-    s.pl = cnd ? 0.f : s.pl;
+    if (FWD) {
+      s.Q = fmaxf(s.Q, m);
+    } else {
+      s.Q = cnd ? m : s.Q;
+      s.pl = cnd ? 0.f : s.pl;
+    }
     float num, den, ki, kc;
     if (FASTOUT) {
       const float he = cp.H * e2;
@@ -840,11 +850,12 @@ __device__ __forceinline__ RevAgg chunk_forward(ChanState& s, const ChanParams& 
 // register pair for the packed output, gate, factor and dr arithmetic, whose lanes round
 // as the scalar forms. The map's sums (lb, lg, lbd, lgd) are kept as even- and odd-token
 // partial sums, added at the end.
-template <bool GATE, bool DR, int RB>
+template <bool GATE, bool DR, int RB, bool FWD>
 __device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanParams& cp, float* K,
                                                       const float* V, float* R, float* DY,
                                                       ChunkFactors& f) {
   static_assert(kTT % RB == 0 && kTT % 2 == 0, "windows and pairs must tile the chunk");
+  static_assert(!FWD || RB >= 2, "a pair must not straddle two windows of the forward's form");
   const float2 l2e = make_float2(kLog2e, kLog2e);
   const float2 w2 = make_float2(cp.w2, cp.w2);
   const float2 H = make_float2(cp.H, cp.H);
@@ -856,9 +867,16 @@ __device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanPa
     const float2 kk = make_float2(K[t * 32], K[(t + 1) * 32]);
     const float2 vv = make_float2(V[t * 32], V[(t + 1) * 32]);
     const float2 gy = make_float2(DY[t * 32], DY[(t + 1) * 32]);
-    // tok_log2w of both tokens: the product rounded on its own, then the fma
-    const float2 m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
-                                __fmul2_rn(kk, l2e));
+    // FWD: the streaming forward's token weights, against the window start (RB >= 2: both
+    // tokens of a pair share it); else tok_log2w of both tokens: the product rounded on its
+    // own, then the fma
+    float2 m;
+    if (FWD)
+      m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
+                     __ffma2_rn(kk, l2e, make_float2(-pl, -pl)));
+    else
+      m = __ffma2_rn(make_float2(float(t % RB + 1), float((t + 1) % RB + 1)), w2,
+                     __fmul2_rn(kk, l2e));
     float2 sig = make_float2(1.f, 1.f);
     if (GATE) {
       const float2 x = __fmul2_rn(make_float2(R[t * 32], R[(t + 1) * 32]),
@@ -871,13 +889,17 @@ __device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanPa
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const float mh = h ? m.y : m.x;
-      const float d = (mh - Q) - pl;
+      const float d = FWD ? mh - Q : (mh - Q) - pl;
       ee[h] = ex2(-fabsf(d));
       const bool cnd = d > 0.f;
       e1s[h] = cnd ? ee[h] : 1.f;
       e2s[h] = cnd ? 1.f : ee[h];
-      Q = cnd ? mh : Q;
-      pl = cnd ? 0.f : pl;
+      if (FWD) {
+        Q = fmaxf(Q, mh);
+      } else {
+        Q = cnd ? mh : Q;
+        pl = cnd ? 0.f : pl;
+      }
       f.tok |= cnd ? (1u << (t + h)) : 0u;
       if ((t + h + 1) % RB == 0) indep_rebase(Q, pl, float(RB) * cp.w2);
     }
@@ -942,18 +964,21 @@ __device__ __forceinline__ RevAgg chunk_forward_pairs(ChanState& s, const ChanPa
   return A;
 }
 
-template <bool GATE, bool DR, bool FASTOUT>
+template <bool GATE, bool DR, bool FASTOUT, bool FWD>
 __device__ __forceinline__ RevAgg chunk_forward_rb(ChanState& s, const ChanParams& cp, int rb,
                                                    float* K, const float* V, float* R, float* DY,
                                                    ChunkFactors& f) {
   if constexpr (FASTOUT) {
-    if (rb == 16) return chunk_forward_pairs<GATE, DR, 16>(s, cp, K, V, R, DY, f);
-    if (rb == 4) return chunk_forward_pairs<GATE, DR, 4>(s, cp, K, V, R, DY, f);
-    return chunk_forward_pairs<GATE, DR, 1>(s, cp, K, V, R, DY, f);
+    if (rb == 16) return chunk_forward_pairs<GATE, DR, 16, FWD>(s, cp, K, V, R, DY, f);
+    if (rb == 4) return chunk_forward_pairs<GATE, DR, 4, FWD>(s, cp, K, V, R, DY, f);
+    if constexpr (FWD)  // windows of one token: each its own window start
+      return chunk_forward<GATE, DR, true, 1, FWD>(s, cp, K, V, R, DY, f);
+    else
+      return chunk_forward_pairs<GATE, DR, 1, FWD>(s, cp, K, V, R, DY, f);
   } else {
-    if (rb == 16) return chunk_forward<GATE, DR, false, 16>(s, cp, K, V, R, DY, f);
-    if (rb == 4) return chunk_forward<GATE, DR, false, 4>(s, cp, K, V, R, DY, f);
-    return chunk_forward<GATE, DR, false, 1>(s, cp, K, V, R, DY, f);
+    if (rb == 16) return chunk_forward<GATE, DR, false, 16, FWD>(s, cp, K, V, R, DY, f);
+    if (rb == 4) return chunk_forward<GATE, DR, false, 4, FWD>(s, cp, K, V, R, DY, f);
+    return chunk_forward<GATE, DR, false, 1, FWD>(s, cp, K, V, R, DY, f);
   }
 }
 
@@ -1049,7 +1074,7 @@ __device__ __forceinline__ float2 chunk_reverse_pairs(const ChunkFactors& f, Rev
 //      over its chunk: dk, dv in place of wkv, v, TMA-stored with dr; warp 0 publishes the
 //      carry at the segment's start where a segment further back starts from it; the
 //      chunks' partial sums of dw, du are added in a fixed order into per-segment partials.
-template <bool GATE, bool DR>
+template <bool GATE, bool DR, bool FWD>
 __global__ void __launch_bounds__(kSW * 32, 5)
     wkv_bwd_seg_kernel(const __grid_constant__ TensorMaps4 in_maps,
                        const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
@@ -1160,8 +1185,8 @@ __global__ void __launch_bounds__(kSW * 32, 5)
     // Past the last token (zero-filled tiles): a weight of 2^{-huge} makes the positions
     // inert (e1 = 1, e2 = 0: the state and the reverse sums pass through unchanged).
     for (int t = nvalid; t < kTT; ++t) K[t * 32] = -1.0e30f;
-    A = fast ? chunk_forward_rb<GATE, DR, true>(s, cp, rb, K, V, R, DY, f)
-             : chunk_forward_rb<GATE, DR, false>(s, cp, rb, K, V, R, DY, f);
+    A = fast ? chunk_forward_rb<GATE, DR, true, FWD>(s, cp, rb, K, V, R, DY, f)
+             : chunk_forward_rb<GATE, DR, false, FWD>(s, cp, rb, K, V, R, DY, f);
     A.L = float(nvalid);  // the inert positions add no distance
   }
   // The carry at this chunk's end comes scaled by the state entering the next chunk (its
@@ -1330,7 +1355,8 @@ int launch_main(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
 template <bool GATE, bool DR>
 int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, int64_t nitems,
                cudaStream_t stream) {
-  auto kern = wkv_bwd_seg_kernel<GATE, DR>;
+  // Checkpoints made by the streaming forward: recompute in its arithmetic.
+  auto kern = a.have_ckpt ? wkv_bwd_seg_kernel<GATE, DR, true> : wkv_bwd_seg_kernel<GATE, DR, false>;
   const size_t smem = size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)

@@ -22,6 +22,35 @@
 
 namespace wkv {
 
+// A full tile of TT tokens for the checkpointing forward: windows of RB tokens, and before
+// each chunk of 16 the state entering it stored at ck[h * stride] (explicitly global, so
+// the store does not order the shared-memory traffic around it).
+template <typename Tin, bool GATE, bool FASTOUT, int TT, int RS, int RB>
+__device__ __forceinline__ void ckpt_tile(ChanState& s, const ChanParams& cp, const Tin* K,
+                                          const Tin* V, const Tin* R, Tin* Y, float4* ck,
+                                          size_t stride, bool valid) {
+#pragma unroll
+  for (int h = 0; h < TT / 16; ++h) {
+    if (valid) __stcg(ck + h * stride, make_float4(s.a, s.b, s.Q, s.pl));
+#pragma unroll
+    for (int w0 = h * 16; w0 < h * 16 + 16; w0 += RB)
+      window_smem<Tin, GATE, FASTOUT, RB, RS>(s, cp, K + w0 * RS, V + w0 * RS, R + w0 * RS,
+                                              Y + w0 * RS);
+  }
+}
+
+template <typename Tin, bool GATE, bool FASTOUT, int TT, int RS>
+__device__ __forceinline__ void ckpt_tile_rb(ChanState& s, const ChanParams& cp, const Tin* K,
+                                             const Tin* V, const Tin* R, Tin* Y, int rb,
+                                             float4* ck, size_t stride, bool valid) {
+  if (rb == 16)
+    ckpt_tile<Tin, GATE, FASTOUT, TT, RS, 16>(s, cp, K, V, R, Y, ck, stride, valid);
+  else if (rb == 4)
+    ckpt_tile<Tin, GATE, FASTOUT, TT, RS, 4>(s, cp, K, V, R, Y, ck, stride, valid);
+  else
+    ckpt_tile<Tin, GATE, FASTOUT, TT, RS, 1>(s, cp, K, V, R, Y, ck, stride, valid);
+}
+
 __device__ __forceinline__ void cta_sync(int nw) {
   if (nw == 1)
     __syncwarp();
@@ -32,12 +61,18 @@ __device__ __forceinline__ void cta_sync(int nw) {
 // Launch bounds: with no minimum, ptxas sizes registers for the 32-CTA residency limit
 // (32 registers at NW = 2), which serialises the windows; residency is bounded by shared
 // memory to a few CTAs per SM anyway, so ask for 4.
-template <typename Tin, bool GATE, int TT, int S, int NW>
+// CKPT (fp32 training forward): also write the state entering every chunk of 16 tokens to
+// ckpt ([B, ceil(T/16), C] float4 (a, b, Q, pl)) and the state after the last token to
+// ckend ([B, C]): the checkpoints of the backward's reverse pass, which recomputes each chunk
+// from them in these same operations. The chunks are processed as separate pieces of 16
+// tokens, which changes nothing: windows never cross a multiple of 16.
+template <typename Tin, bool GATE, int TT, int S, int NW, bool CKPT = false>
 __global__ void __launch_bounds__(NW * 32, 4) wkv_fwd_tma_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_y, int T,
     int C, const float* __restrict__ w, const float* __restrict__ u, const float* a0,
-    const float* b0, const float* p0, float* a1, float* b1, float* p1, unsigned* err) {
+    const float* b0, const float* p0, float* a1, float* b1, float* p1, unsigned* err,
+    float4* ckpt, float4* ckend) {
   // Full tiles are processed in whole windows of up to 16 tokens.
   static_assert(TT % 16 == 0, "tile length must be a multiple of the longest window");
   static_assert(S >= 2, "the y staging wait below assumes two or more stages");
@@ -97,7 +132,37 @@ __global__ void __launch_bounds__(NW * 32, 4) wkv_fwd_tma_kernel(
     const Tin* R = sr + st * kTile + tid;
     Tin* Y = sy + st * kTile + tid;
     const int n = min(TT, T - i * TT);
-    if (n == TT) {
+    if (CKPT && n == TT) {
+      float4* ck = ckpt + (size_t(b) * ((T + 15) / 16) + size_t(i) * (TT / 16)) * C + c;
+      if (fast)
+        ckpt_tile_rb<Tin, GATE, true, TT, CW>(s, cp, K, V, R, Y, rb, ck, size_t(C), valid);
+      else
+        ckpt_tile_rb<Tin, GATE, false, TT, CW>(s, cp, K, V, R, Y, rb, ck, size_t(C), valid);
+    } else if (CKPT) {  // the last, partial tile: chunk by chunk
+      const int nch = (T + 15) / 16;
+#pragma unroll
+      for (int h = 0; h < TT / 16; ++h) {
+        if (h * 16 < n) {
+          if (valid)
+            ckpt[(size_t(b) * nch + size_t(i) * (TT / 16) + h) * C + c] =
+                make_float4(s.a, s.b, s.Q, s.pl);
+          const int o = h * 16 * CW;
+          const int nq = min(16, n - h * 16);
+          if (nq == 16) {
+            if (fast)
+              full_tile<Tin, GATE, true, 16, CW>(s, cp, K + o, V + o, R + o, Y + o, rb);
+            else
+              full_tile<Tin, GATE, false, 16, CW>(s, cp, K + o, V + o, R + o, Y + o, rb);
+          } else if (fast) {
+            tile_tokens<Tin, GATE, true, 16, 1, CW, false>(s, cp, K + o, V + o, R + o, Y + o,
+                                                          nq, rb);
+          } else {
+            tile_tokens<Tin, GATE, false, 16, 1, CW, false>(s, cp, K + o, V + o, R + o, Y + o,
+                                                           nq, rb);
+          }
+        }
+      }
+    } else if (n == TT) {
       if (fast)
         full_tile<Tin, GATE, true, TT, CW>(s, cp, K, V, R, Y, rb);
       else
@@ -120,6 +185,7 @@ __global__ void __launch_bounds__(NW * 32, 4) wkv_fwd_tma_kernel(
     }
   }
   if (tid == 0) tma_store_wait_all();
+  if (CKPT && valid) ckend[sidx] = make_float4(s.a, s.b, s.Q, s.pl);
 
   if (a1 != nullptr && valid) {
     a1[sidx] = s.a;
@@ -210,8 +276,9 @@ size_t tma_smem_bytes() {
          F::S * sizeof(uint64_t);
 }
 
-template <typename Tin, bool GATE>
-int launch_tma(const FwdArgs& a, cudaStream_t stream) {
+template <typename Tin, bool GATE, bool CKPT = false>
+int launch_tma(const FwdArgs& a, cudaStream_t stream, float4* ckpt = nullptr,
+               float4* ckend = nullptr) {
   using F = FwdCfg<Tin>;
   constexpr int CW = F::NW * 32;
   CUtensorMap tk, tv, tr, ty;
@@ -222,7 +289,7 @@ int launch_tma(const FwdArgs& a, cudaStream_t stream) {
   if (!rc) rc = encode_btc_map(&tr, GATE ? a.r : a.k, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
   if (!rc) rc = encode_btc_map(&ty, a.y, dt, sizeof(Tin), a.B, a.T, a.C, CW, F::TT);
   if (rc) return rc;
-  auto kern = wkv_fwd_tma_kernel<Tin, GATE, F::TT, F::S, F::NW>;
+  auto kern = wkv_fwd_tma_kernel<Tin, GATE, F::TT, F::S, F::NW, CKPT>;
   const size_t smem = tma_smem_bytes<Tin, GATE>();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
@@ -230,7 +297,7 @@ int launch_tma(const FwdArgs& a, cudaStream_t stream) {
   const int64_t G = (a.C + CW - 1) / CW;
   const int64_t grid = a.B * G;
   kern<<<unsigned(grid), CW, smem, stream>>>(tk, tv, tr, ty, int(a.T), int(a.C), a.w, a.u, a.a0,
-                                             a.b0, a.p0, a.a1, a.b1, a.p1, a.err);
+                                             a.b0, a.p0, a.a1, a.b1, a.p1, a.err, ckpt, ckend);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -259,6 +326,15 @@ bool fwd_tma_ok(const FwdArgs& a, int elem_bytes) {
   return (a.C * elem_bytes) % 16 == 0 && al16(a.k) && al16(a.v) && al16(a.r) && al16(a.y) &&
          a.T < (int64_t(1) << 31) && a.C < (int64_t(1) << 31) && a.B < (int64_t(1) << 31) &&
          a.B * ((a.C + 31) / 32) < (int64_t(1) << 31);
+}
+
+int launch_fwd_ckpt(const FwdArgs& a, void* ws, cudaStream_t stream) {
+  static_assert(FwdCfg<float>::NW == 1, "checkpoints are made per warp of 32 channels");
+  if (!fwd_tma_ok(a, 4)) return WKV_ERR_UNSUPPORTED;
+  float4 *ckpt = nullptr, *ckend = nullptr;
+  backward_checkpoint_ptrs(ws, a.B, a.T, a.C, &ckpt, &ckend);
+  return a.r != nullptr ? launch_tma<float, true, true>(a, stream, ckpt, ckend)
+                        : launch_tma<float, false, true>(a, stream, ckpt, ckend);
 }
 
 int launch_fwd_stream(const FwdArgs& a, bool bf16, bool force_plain, cudaStream_t stream) {

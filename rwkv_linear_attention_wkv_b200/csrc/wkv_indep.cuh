@@ -1,16 +1,17 @@
-// The per-token scale step with a state-independent token weight, shared by every kernel
-// whose states must agree bit for bit with the backward's recomputation: the checkpoint
-// pass and the reverse pass of the backward (wkv_bwd.cu) and the checkpointing training
-// forward (wkv_fwd_ckpt.cu).
+// The per-token scale step with a state-independent token weight, used by the backward's
+// checkpoint pass and by its reverse pass when it recomputes from that pass's checkpoints
+// (wkv_bwd.cu).
 //
-// A checkpoint is a state (a, b, Q, pl) at a chunk boundary; the reverse pass recomputes the
-// chunk from it. Both sides must weigh every token identically, or a dominant token (a spike
-// in k) would carry two different roundings of its weight into the two sides and the
-// reverse sums would be inconsistent at the level of ulp(k log2 e). So the token's
-// log2-weight in the window, m = k log2(e) + j w2, is rounded independently of the state,
-// and the state's low part enters only the comparison d = (m - Q) - pl; a token that takes
-// over the scale sets it to (m, 0). (The streaming forward of wkv_step.cuh folds pl into m
-// instead and keeps Q as a running maximum: the same quantity, rounded differently.)
+// Those checkpoints are formed by combining chunk aggregates (not by walking the tokens),
+// and the reverse pass recomputes each chunk from one. Both sides must weigh every token
+// identically, or a dominant token (a spike in k) would carry two different roundings of
+// its weight into the two sides and the reverse sums would be inconsistent at the level of
+// ulp(k log2 e). So the token's log2-weight in the window, m = k log2(e) + j w2, is rounded
+// independently of the state, and the state's low part enters only the comparison
+// d = (m - Q) - pl; a token that takes over the scale sets it to (m, 0). (The streaming
+// forward of wkv_step.cuh folds pl into m instead and keeps Q as a running maximum: the
+// same quantity, rounded differently. Checkpoints that the streaming forward writes are
+// recomputed in that form.)
 #pragma once
 
 #include "wkv_step.cuh"

@@ -105,7 +105,8 @@ struct BwdArgs {
   unsigned long long wait_ns = 2000000000ull;
   int withhold_last_map = 0;
   // The workspace already holds the checkpoints (written by launch_fwd_ckpt over the same
-  // w, k, v and initial state): the checkpoint pass is skipped. Time-parallel path only.
+  // w, k, v and initial state): the checkpoint pass is skipped and the reverse pass
+  // recomputes in the streaming forward's arithmetic. Time-parallel path only.
   int have_ckpt = 0;
 };
 size_t backward_workspace_bytes(int64_t B, int64_t T, int64_t C);
@@ -117,8 +118,8 @@ void backward_checkpoint_ptrs(void* ws, int64_t B, int64_t T, int64_t C, float4*
 // Whether the backward takes its time-parallel (checkpointed) path for these arguments.
 bool backward_time_parallel_ok(const BwdArgs& a);
 // Forward (fp32, TMA shapes only: else WKV_ERR_UNSUPPORTED) that also writes the backward's
-// checkpoints into its workspace ws, in the arithmetic of the backward's recomputation
-// (wkv_fwd_ckpt.cu).
+// checkpoints into its workspace ws: the streaming kernel in its checkpointing mode
+// (wkv_fwd.cu); a backward with have_ckpt set recomputes in the same arithmetic.
 int launch_fwd_ckpt(const FwdArgs& a, void* ws, cudaStream_t stream);
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);
 // T == 0 with the state's gradients wanted: they pass straight through.

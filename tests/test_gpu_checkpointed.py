@@ -151,6 +151,8 @@ def test_checkpointed_pair_training_shape_and_determinism(W):
     g3 = W.wkv_backward_checkpointed(w, u, k, v, r, dev(x.dy), ws)  # the workspace is reused
     assert W.wkv_stream_status() == 0
     assert torch.equal(y1, y2)
+    # the streaming kernel of wkv_forward (B * C = 12288 channels), checkpoints aside
+    assert torch.equal(y2, W.wkv_forward(w, u, k, v, r))
     for n in ("dk", "dv", "dr", "dw", "du"):
         assert torch.equal(g1[n], g2[n]), n
         assert torch.equal(g2[n], g3[n]), n
