@@ -95,6 +95,18 @@ def test_backward_time_parallel_segments(W, shape):
     check(W, x)
 
 
+@pytest.mark.parametrize("shape", [(3, 150, 2752), (1, 67, 8192), (2, 33, 4100)])
+@pytest.mark.parametrize("gate", [True, False])
+def test_backward_many_channels(W, shape, gate):
+    # Thousands of channels with k spikes and decays from e^-6 to e^2: many independent
+    # 32-channel groups per segment, ragged T (a partial last chunk) and a partial group
+    # (C = 4100).
+    B, T, C = shape
+    x = wkv_inputs.make_inputs(B, T, C, seed=C + T, logw_range=(-6, 2), u_bound=2.0,
+                               k_std=3.0, spike_frac=1e-3, with_dy=True)
+    check(W, x, gate)
+
+
 def test_backward_workspace_checks(W):
     import ctypes
     x = wkv_inputs.make_inputs(1, 10, 8, seed=1, with_dy=True)

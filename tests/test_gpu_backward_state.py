@@ -92,6 +92,18 @@ def test_backward_state_one_side_only(W, with_state, with_grad):
     run(W, x, *make_state(2, 64, 5), with_state=with_state, with_grad=with_grad)
 
 
+@pytest.mark.parametrize("shape", [(2, 97, 4096), (3, 40, 2752)])
+def test_backward_state_many_channels(W, shape):
+    # Thousands of channels with a state on both sides, the inputs of the shapes test. (With
+    # k spikes added, one dv element of 794,624 at 2 x 97 x 4096 lands at 1.03 times the
+    # elementwise bound 1e-5 (1 + |ref|), the same on the time-parallel and the serial
+    # checkpoint paths: dv is a sum whose terms cancel there, and the bound does not scale
+    # with the terms.)
+    B, T, C = shape
+    x = wkv_inputs.make_inputs(B, T, C, seed=T + C, k_std=2.0, with_dy=True)
+    run(W, x, *make_state(B, C, T))
+
+
 def test_backward_state_spikes(W):
     x = wkv_inputs.make_inputs(2, 300, 64, seed=8, logw_range=(-6, 2), u_bound=2.0, k_std=3.0,
                                spike_frac=0.01, with_dy=True)
