@@ -9,15 +9,14 @@
 // The report gives no read-out; this library reads the state with the receptance as the
 // query, y_t = S_t r_t^T.
 //
-// One CTA per (batch row, head) of head size N = 64, 64 threads: thread t holds the 8 x 8
-// block of S at rows 8 (t / 8) .., columns {16 m + 2 (t mod 8), 16 m + 2 (t mod 8) + 1 : m < 4}
+// One CTA per (batch row, head) of head size N = 64, 64 threads: thread t holds the 4 x 16
+// block of S at rows 4 (t / 4) .., columns {8 m + 2 (t mod 4), 8 m + 2 (t mod 4) + 1 : m < 8}
 // in registers, as pairs for packed fp32x2 arithmetic. A token's vectors are read from
-// shared memory once per thread (64-byte
-// contiguous, conflict-free 8-byte reads, shared by broadcast between row blocks) instead
-// of once per row, which keeps the shared-memory traffic per token at about 1.5 KB per
-// warp. Row sums (sa_i = S[i] . a and y_i = S[i] . r) reduce over the 8 threads of a row
-// block by recursive halving (7 shuffles for 8 rows), and sa is gathered back the same
-// way. r, w, k, v, a, b ([64] fp32 each per token) come in TMA tiles of kT7 tokens through
+// shared memory once per thread (conflict-free 8-byte reads, 32 contiguous bytes per
+// instruction, shared by broadcast between row blocks) instead of once per row. Row sums
+// (sa_i = S[i] . a and y_i = S[i] . r) reduce over the 4 threads of a row block by
+// recursive halving (3 shuffles for 4 rows; 8 x 8 blocks over 8 threads took 7 for 8 rows
+// and measured 5% slower), and sa is gathered back the same way. r, w, k, v, a, b ([64] fp32 each per token) come in TMA tiles of kT7 tokens through
 // a kS7-stage mbarrier pipeline; y is staged in shared memory and TMA-stored a tile at a
 // time. Bound: the FP32 pipe (about 5 N^2 operations per token per head).
 #include "wkv_device.cuh"
@@ -30,37 +29,35 @@ namespace {
 constexpr int kN7 = 64;        // head size
 constexpr int kT7 = 8;         // tokens per tile
 constexpr int kS7 = 4;         // pipeline stages
-constexpr int kBR = 8;         // rows of S per thread
-constexpr int kBC = 8;         // columns of S per thread (4 pairs, 16 columns apart)
-constexpr int kThr7 = (kN7 / kBR) * (kN7 / kBC);  // threads per head (64)
+constexpr int kBR = 4;         // rows of S per thread
+constexpr int kBC = 16;        // columns of S per thread (kPr pairs, 2 kLB columns apart)
+constexpr int kPr = kBC / 2;   // column pairs per thread
+constexpr int kLB = kN7 / kBC; // lanes of a row block (threads sharing its rows)
+constexpr int kThr7 = (kN7 / kBR) * kLB;  // threads per head (64)
+static_assert(kBR == kLB, "the row reductions halve rows and lanes together");
 constexpr int kTile7 = kT7 * kN7;  // floats per tensor tile
 
 struct Wkv7Maps {
   CUtensorMap r, w, k, v, a, b, y;
 };
 
-// Sum over the 8 lanes of a row block (lanes 8m .. 8m+7) of x[r] for each of the kBR rows:
-// recursive halving (exchange half the rows with the lane differing in bit 2, then bit 1,
-// ...) and, once one row is left, a butterfly sum. Lane l ends with the full sum for row
-// (l mod 8) >> (3 - log2 kBR) of the block.
+// Sum over the kLB lanes of a row block of x[r] for each of its kBR (= kLB) rows: recursive
+// halving (exchange half the rows with the lane differing in the highest bit of the block,
+// then the next, ...). Lane l ends with the full sum for row l mod kLB of the block.
 __device__ __forceinline__ float rowblock_reduce(float (&x)[kBR], int lc) {
   int half = kBR / 2;
 #pragma unroll
-  for (int bit = 4; bit >= 1; bit >>= 1) {
-    if (half >= 1) {
-      const bool up = lc & bit;
+  for (int bit = kLB / 2; bit >= 1; bit >>= 1) {
+    const bool up = lc & bit;
 #pragma unroll
-      for (int r = 0; r < kBR / 2; ++r) {
-        if (r < half) {
-          const float send = up ? x[r] : x[r + half];
-          const float got = __shfl_xor_sync(0xffffffffu, send, bit);
-          x[r] = (up ? x[r + half] : x[r]) + got;
-        }
+    for (int r = 0; r < kBR / 2; ++r) {
+      if (r < half) {
+        const float send = up ? x[r] : x[r + half];
+        const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+        x[r] = (up ? x[r + half] : x[r]) + got;
       }
-      half >>= 1;
-    } else {
-      x[0] += __shfl_xor_sync(0xffffffffu, x[0], bit);
     }
+    half >>= 1;
   }
   return x[0];
 }
@@ -70,25 +67,20 @@ __device__ __forceinline__ void rowblock_reduce2(float (&x)[kBR], float (&z)[kBR
                                                  float& xs, float& zs) {
   int half = kBR / 2;
 #pragma unroll
-  for (int bit = 4; bit >= 1; bit >>= 1) {
-    if (half >= 1) {
-      const bool up = lc & bit;
+  for (int bit = kLB / 2; bit >= 1; bit >>= 1) {
+    const bool up = lc & bit;
 #pragma unroll
-      for (int r = 0; r < kBR / 2; ++r) {
-        if (r < half) {
-          const float sx = up ? x[r] : x[r + half];
-          const float sz = up ? z[r] : z[r + half];
-          const float gx = __shfl_xor_sync(0xffffffffu, sx, bit);
-          const float gz = __shfl_xor_sync(0xffffffffu, sz, bit);
-          x[r] = (up ? x[r + half] : x[r]) + gx;
-          z[r] = (up ? z[r + half] : z[r]) + gz;
-        }
+    for (int r = 0; r < kBR / 2; ++r) {
+      if (r < half) {
+        const float sx = up ? x[r] : x[r + half];
+        const float sz = up ? z[r] : z[r + half];
+        const float gx = __shfl_xor_sync(0xffffffffu, sx, bit);
+        const float gz = __shfl_xor_sync(0xffffffffu, sz, bit);
+        x[r] = (up ? x[r + half] : x[r]) + gx;
+        z[r] = (up ? z[r + half] : z[r]) + gz;
       }
-      half >>= 1;
-    } else {
-      x[0] += __shfl_xor_sync(0xffffffffu, x[0], bit);
-      z[0] += __shfl_xor_sync(0xffffffffu, z[0], bit);
     }
+    half >>= 1;
   }
   xs = x[0];
   zs = z[0];
@@ -105,13 +97,13 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
   __shared__ uint64_t bars[kS7];
   const int tid = threadIdx.x;
   const int lane = tid & 31;
-  const int lc = tid & 7;          // column block (and, after a row reduction, the row)
-  const int r0 = (tid >> 3) * kBR;  // first row of this thread's block
+  const int lc = tid & (kLB - 1);    // column block (and, after a row reduction, the row)
+  const int r0 = (tid / kLB) * kBR;  // first row of this thread's block
   const int bh = blockIdx.x;
   const int b = bh / H, h = bh - b * H;
   const int ntile = (T + kT7 - 1) / kT7;
-  // column of pair m (0..3), element e (0..1) of this thread
-  auto col = [&](int m, int e) { return 16 * m + 2 * lc + e; };
+  // column of pair m (0 .. kPr-1), element e (0..1) of this thread
+  auto col = [&](int m, int e) { return 2 * kLB * m + 2 * lc + e; };
 
   auto issue = [&](int st, int tile) {
     uint64_t* bar = &bars[st];
@@ -132,13 +124,13 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
   }
   __syncthreads();
 
-  float2 S[kBR][kBC / 2];  // S[r][m] = state[r0 + r][col(m, 0 .. 1)]
+  float2 S[kBR][kPr];  // S[r][m] = state[r0 + r][col(m, 0 .. 1)]
   {
     const float* src = s0 ? s0 + (size_t(bh) * kN7 + r0) * kN7 : nullptr;
 #pragma unroll
     for (int r = 0; r < kBR; ++r)
 #pragma unroll
-      for (int m = 0; m < 4; ++m)
+      for (int m = 0; m < kPr; ++m)
         S[r][m] = src ? *reinterpret_cast<const float2*>(src + r * kN7 + col(m, 0))
                       : make_float2(0.f, 0.f);
   }
@@ -162,20 +154,20 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
       for (int r = 0; r < kBR; ++r) {
         float2 p = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < 4; ++m)
+        for (int m = 0; m < kPr; ++m)
           p = __ffma2_rn(S[r][m], *reinterpret_cast<const float2*>(tok + 4 * kTile7 + col(m, 0)), p);
         part[r] = p.x + p.y;
       }
     }
-    float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc / (8 / kBR)
+    float sa_mine = rowblock_reduce(part, lc);  // sa for row r0 + lc
 #pragma unroll 1
     for (int t = 0; t < n; ++t) {
       const float* tok = base + t * kN7;
       const bool next = t + 1 < n;
       // the token's vectors at this thread's columns (pairs), and v at its rows
-      float2 rv[4], wv[4], kv[4], bv[4], an[4];
+      float2 rv[kPr], wv[kPr], kv[kPr], bv[kPr], an[kPr];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
+      for (int m = 0; m < kPr; ++m) {
         rv[m] = *reinterpret_cast<const float2*>(tok + 0 * kTile7 + col(m, 0));
         wv[m] = *reinterpret_cast<const float2*>(tok + 1 * kTile7 + col(m, 0));
         kv[m] = *reinterpret_cast<const float2*>(tok + 2 * kTile7 + col(m, 0));
@@ -193,12 +185,12 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
       // token's sa_i = S_t[i] . a_{t+1}
 #pragma unroll
       for (int r = 0; r < kBR; ++r) {
-        const float sr = __shfl_sync(0xffffffffu, sa_mine, (lane & ~7) | (r * (8 / kBR)));
+        const float sr = __shfl_sync(0xffffffffu, sa_mine, (lane & ~(kLB - 1)) | r);
         const float2 sa2 = make_float2(sr, sr);
         const float2 v2 = make_float2(vv[r], vv[r]);
         float2 p = make_float2(0.f, 0.f), q = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
+        for (int m = 0; m < kPr; ++m) {
           S[r][m] = __ffma2_rn(S[r][m], wv[m], __ffma2_rn(sa2, bv[m], __fmul2_rn(v2, kv[m])));
           p = __ffma2_rn(S[r][m], rv[m], p);
           q = __ffma2_rn(S[r][m], an[m], q);
@@ -212,7 +204,7 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
       } else {
         y_mine = rowblock_reduce(part, lc);
       }
-      if (lc % (8 / kBR) == 0) yt[t * kN7 + r0 + lc / (8 / kBR)] = y_mine;
+      yt[t * kN7 + r0 + lc] = y_mine;
     }
     fence_proxy_async_smem();  // the y tile's writes, visible to the TMA store
     __syncthreads();           // the stage is consumed and the y tile complete
@@ -227,7 +219,7 @@ __global__ void __launch_bounds__(kThr7) wkv7_fwd_kernel(const __grid_constant__
 #pragma unroll
     for (int r = 0; r < kBR; ++r)
 #pragma unroll
-      for (int m = 0; m < 4; ++m) *reinterpret_cast<float2*>(dst + r * kN7 + col(m, 0)) = S[r][m];
+      for (int m = 0; m < kPr; ++m) *reinterpret_cast<float2*>(dst + r * kN7 + col(m, 0)) = S[r][m];
   }
   if (tid == 0) tma_store_wait_all();
 }
