@@ -61,7 +61,9 @@ typedef enum wkv_status {
   WKV_ERR_ALIGNMENT = 2,   /* a pointer not aligned to its element size                */
   WKV_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed              */
   WKV_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (wkv_stream_status)   */
-  WKV_ERR_UNSUPPORTED = 5, /* a size beyond what the kernels index (e.g. T >= 2^31)    */
+  WKV_ERR_UNSUPPORTED = 5, /* a size beyond what the kernels index (e.g. T >= 2^31), or
+                              a shape an entry point's kernels cannot take (documented
+                              with the entry point)                                       */
   WKV_ERR_SCRATCH_LIMIT = 6 /* wkv_forward_state_static: the problem needs more scratch
                                than the library's fixed array holds                       */
 } wkv_status;
@@ -69,7 +71,8 @@ typedef enum wkv_status {
 /* Human-readable name of a status code. Never NULL. */
 WKV_API const char* wkv_status_string(int status);
 
-/* Library ABI version (major * 10000 + minor * 100 + patch). */
+/* Library ABI version (major * 10000 + minor * 100 + patch). 1.1: the checkpointed
+ * training pair (wkv_forward_checkpointed, wkv_backward_checkpointed). */
 WKV_API int wkv_version(void);
 
 /*

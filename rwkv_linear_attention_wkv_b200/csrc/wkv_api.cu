@@ -229,7 +229,7 @@ WKV_API const char* wkv_status_string(int status) {
   }
 }
 
-WKV_API int wkv_version(void) { return 10000; }
+WKV_API int wkv_version(void) { return 10100; }
 
 WKV_API int wkv_forward(int64_t B, int64_t T, int64_t C, const float* w, const float* u,
                         const float* k, const float* v, const float* r, float* y,
