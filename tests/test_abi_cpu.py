@@ -138,3 +138,37 @@ def test_checkpointed_pair_argument_checks(W):
     assert bc(2, 64, 32, *base, [ok, None, ok][0], None, ok, *none3, *outs, *none3, ok, need,
               None) == 1
     assert bc(0, 64, 32, *base, *none3, *none3, *outs, *none3, ok, need, None) == 0
+
+
+def declared_signatures():
+    """{name: [parameter types]} of every WKV_API function in include/*.h."""
+    sigs = {}
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = re.sub(r"/\*.*?\*/", " ", open(os.path.join(ROOT, "include", h)).read(), flags=re.S)
+        for m in re.finditer(r"WKV_API\s+[\w\s\*]+?\b(\w+)\s*\(([^)]*)\)\s*;", text):
+            params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+            sigs[m.group(1)] = [re.sub(r"\s+\w+$", "", p) for p in params]
+    return sigs
+
+
+def test_binding_matches_the_declarations(W):
+    # Every function the binding types matches its declaration parameter for parameter:
+    # 64-bit sizes, ints, size_t and pointers (including the stream) where the header has them.
+    from rwkv_linear_attention_wkv_b200 import _SIGS
+    sigs = declared_signatures()
+    # (size_t and uint64_t are the same 64-bit unsigned type on this ABI, as are their
+    # ctypes names)
+    kinds = {ctypes.c_int64: "i64", ctypes.c_int: "int", ctypes.c_size_t: "u64",
+             ctypes.c_uint64: "u64", ctypes.c_void_p: "ptr"}
+
+    def kind(t):
+        t = t.replace("const ", "").strip()
+        if t.endswith("*") or t == "cudaStream_t":
+            return "ptr"
+        return {"int64_t": "i64", "int": "int", "size_t": "u64", "uint64_t": "u64"}[t]
+
+    for name, (args, _) in _SIGS.items():
+        assert name in sigs, name
+        assert [kinds[a] for a in args] == [kind(t) for t in sigs[name]], name
