@@ -25,18 +25,23 @@
 // sums of |dy sigmoid(r) / den|: no exponential in the reverse pass, nothing to overflow,
 // and the scale is the forward's exact windowed one, so nothing drifts.
 //
-// Two kernels plus a reduction:
-//   1. checkpoint: one warp per 32 channels streams k, v forward (TMA) and stores the
-//      state entering every chunk of kTT tokens;
+// Two passes plus a reduction:
+//   1. checkpoints: the state entering every chunk of kTT tokens. Time-parallel on TMA
+//      shapes (wkv_bwd_ckpt_seg_kernel: chunk aggregates folded across segments, in the
+//      state-independent token weights of wkv_indep.cuh); serially otherwise
+//      (wkv_bwd_ckpt_kernel: one warp per 32 channels walks the sequence in the streaming
+//      forward's arithmetic). In the checkpointed training pair the forward has written
+//      them already (the streaming kernel's checkpointing mode) and this pass is skipped;
 //   2. reverse, time-parallel (TMA shapes): one warp per chunk recomputes the chunk's
-//      forward from its checkpoint, the carries of the reverse sums are chained across
-//      segments of kSW chunks, and each warp then runs the reverse over its chunk (see
-//      section 2' below). Shapes TMA cannot address take the serial form: one warp per 32
-//      channels walks the chunks from last to first, recomputing each chunk's factors into
-//      shared memory before its reverse;
+//      forward from its checkpoint (in the arithmetic that made the checkpoint: the
+//      template flag FWD), the carries of the reverse sums are chained across segments of
+//      kSW chunks, and each warp then runs the reverse over its chunk (see section 2'
+//      below). Shapes TMA cannot address take the serial form: one warp per 32 channels
+//      walks the chunks from last to first, recomputing each chunk's factors into shared
+//      memory before its reverse;
 //   both write dk, dv (dr) in place of k, v (r) in shared memory for the stores, and
-//   per-(b, chunk, c) partial sums of dw, du to the workspace;
-//   3. reduce: dw[c], du[c] = sums of the per-chunk partials over b and t in a fixed order
+//   per-(b, segment or chunk, c) partial sums of dw, du to the workspace;
+//   3. reduce: dw[c], du[c] = sums of the partials over b and t in a fixed order
 //      (deterministic).
 #include <algorithm>
 
