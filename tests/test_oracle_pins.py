@@ -425,3 +425,48 @@ def test_wkv7_split_with_state_handover():
                                    b[:, T1:], S1, want_state=True)
     np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(S2, ST, rtol=1e-13, atol=1e-13)
+
+
+def _wkv7_chunked(r, w, k, v, a, b, S0, L):
+    """One head's recurrence in the chunked (triangular-solve) form, fp64: within a chunk,
+    with gamma_t = w_1 ... w_t per key channel, the decay-normalised state is S_0 plus rank-one
+    terms x_s (b_s / gamma_s)^T + v_s (k_s / gamma_s)^T, where x_t = S_{t-1} a_t solves a
+    unit-triangular system over the chunk's tokens. A different algorithm from the token
+    loop (no state update per token), so it pins the oracle's indexing and transposes."""
+    T, N = k.shape
+    S = S0.copy()
+    y = np.empty((T, N))
+    for c0 in range(0, T, L):
+        n = min(L, T - c0)
+        sl = slice(c0, c0 + n)
+        gam = np.cumprod(w[sl], axis=0)                  # gamma_t, t = 1 .. n
+        gprev = np.vstack([np.ones((1, N)), gam[:-1]])   # gamma_{t-1}
+        at, bt, kt, rt = gprev * a[sl], b[sl] / gam, k[sl] / gam, gam * r[sl]
+        V = v[sl]
+        X = np.zeros((n, N))
+        for t in range(n):                               # forward substitution
+            X[t] = S @ at[t] + sum(X[s] * (bt[s] @ at[t]) + V[s] * (kt[s] @ at[t])
+                                   for s in range(t))
+        for t in range(n):
+            y[c0 + t] = S @ rt[t] + sum(X[s] * (bt[s] @ rt[t]) + V[s] * (kt[s] @ rt[t])
+                                        for s in range(t + 1))
+        g = gam[-1]
+        S = S * g[None, :] + sum(np.outer(X[s], g * bt[s]) + np.outer(V[s], g * kt[s])
+                                 for s in range(n))
+    return y, S
+
+
+@pytest.mark.parametrize("L", [1, 4, 8])
+def test_wkv7_matches_the_chunked_form(L):
+    # Generic inputs (a, b not tied to k), decays in (0.5, 1], a ragged last chunk.
+    g = np.random.Generator(np.random.PCG64(45))
+    B, T, H, N = 1, 19, 2, 6
+    r, k, v, a, b = (g.standard_normal((B, T, H, N)) * 0.5 for _ in range(5))
+    w = g.uniform(0.5, 1.0, (B, T, H, N))
+    S0 = g.standard_normal((B, H, N, N))
+    y, ST = oracle.wkv7_recurrent(r, w, k, v, a, b, S0, want_state=True)
+    for h in range(H):
+        yc, Sc = _wkv7_chunked(r[0, :, h], w[0, :, h], k[0, :, h], v[0, :, h], a[0, :, h],
+                               b[0, :, h], S0[0, h], L)
+        np.testing.assert_allclose(y[0, :, h], yc, rtol=1e-10, atol=1e-10)
+        np.testing.assert_allclose(ST[0, h], Sc, rtol=1e-10, atol=1e-10)
