@@ -54,8 +54,8 @@ def _load():
         lib.oracle_wkv_direct.argtypes = [I, I, I] + [P] * 8
         lib.oracle_wkv_recurrent.argtypes = [I, I, I] + [P] * 10
         lib.oracle_wkv_decode.argtypes = [I, I, I] + [P] * 8
-        lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 13
-        lib.oracle_wkv_backward_state.argtypes = [I, I, I] + [P] * 21
+        lib.oracle_wkv_backward.argtypes = [I, I, I] + [P] * 15
+        lib.oracle_wkv_backward_state.argtypes = [I, I, I] + [P] * 23
         lib.oracle_wkv7_recurrent.argtypes = [I, I, I, I] + [P] * 9
         for f in (lib.oracle_wkv_direct, lib.oracle_wkv_recurrent, lib.oracle_wkv_decode,
                   lib.oracle_wkv_backward, lib.oracle_wkv_backward_state,
@@ -116,7 +116,7 @@ def wkv_decode(w, u, k, v, r, A, Bd):
 
 def wkv_backward(w, u, k, v, r, dy):
     """Analytic fp64 gradients. Returns dict dk, dv, dw, du, dr (dr None if r is None),
-    and dw_abs, du_abs: the sums of |term| behind dw and du."""
+    and dw_abs, du_abs, dk_abs, dv_abs: the sums of |term| behind dw, du, dk and dv."""
     w, u, k, v, r, dy = map(_f64, (w, u, k, v, r, dy))
     B, T, C = k.shape
     dk = np.empty((B, T, C))
@@ -126,17 +126,21 @@ def wkv_backward(w, u, k, v, r, dy):
     du = np.empty(C)
     dwa = np.empty(C)
     dua = np.empty(C)
+    dka = np.empty((B, T, C))
+    dva = np.empty((B, T, C))
     _check(_load().oracle_wkv_backward(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
                                        _ptr(dy), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du),
-                                       _ptr(dr), _ptr(dwa), _ptr(dua)))
-    return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dw_abs": dwa, "du_abs": dua}
+                                       _ptr(dr), _ptr(dwa), _ptr(dua), _ptr(dka), _ptr(dva)))
+    return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dw_abs": dwa, "du_abs": dua,
+            "dk_abs": dka, "dv_abs": dva}
 
 
 def wkv_backward_state(w, u, k, v, r, dy, A0=None, B0=None, gA=None, gB=None):
     """Gradients of sum(dy * y) + sum(gA * A_T) + sum(gB * B_T) for the forward from the
     true initial state (A0, B0) [B, C] (None: empty), by the step-by-step adjoint of the
     recurrence. Returns dict dk, dv, dw, du, dr (None if r is None), dA0, dB0 [B, C], and
-    dw_abs, du_abs, dA0_abs, dB0_abs: the same sums run on absolute values."""
+    dw_abs, du_abs, dA0_abs, dB0_abs, dk_abs, dv_abs: the same sums run on absolute
+    values."""
     w, u, k, v, r, dy, A0, B0, gA, gB = map(_f64, (w, u, k, v, r, dy, A0, B0, gA, gB))
     B, T, C = k.shape
     dk = np.empty((B, T, C))
@@ -144,12 +148,15 @@ def wkv_backward_state(w, u, k, v, r, dy, A0=None, B0=None, gA=None, gB=None):
     dr = np.empty((B, T, C)) if r is not None else None
     dw, du, dwa, dua = (np.empty(C) for _ in range(4))
     dA0, dB0, dA0a, dB0a = (np.empty((B, C)) for _ in range(4))
+    dka = np.empty((B, T, C))
+    dva = np.empty((B, T, C))
     _check(_load().oracle_wkv_backward_state(
         B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(dy), _ptr(A0), _ptr(B0),
         _ptr(gA), _ptr(gB), _ptr(dk), _ptr(dv), _ptr(dw), _ptr(du), _ptr(dr), _ptr(dA0),
-        _ptr(dB0), _ptr(dwa), _ptr(dua), _ptr(dA0a), _ptr(dB0a)))
+        _ptr(dB0), _ptr(dwa), _ptr(dua), _ptr(dA0a), _ptr(dB0a), _ptr(dka), _ptr(dva)))
     return {"dk": dk, "dv": dv, "dw": dw, "du": du, "dr": dr, "dA0": dA0, "dB0": dB0,
-            "dw_abs": dwa, "du_abs": dua, "dA0_abs": dA0a, "dB0_abs": dB0a}
+            "dw_abs": dwa, "du_abs": dua, "dA0_abs": dA0a, "dB0_abs": dB0a,
+            "dk_abs": dka, "dv_abs": dva}
 
 
 def wkv7_recurrent(r, w, k, v, a, b, S0=None, want_state=False):

@@ -149,11 +149,19 @@ int oracle_wkv_decode(int64_t N, int64_t L, int64_t C, const double *w, const do
  *   dw = -sum_{i<t} (t-1-i) e^{k_i-(t-1-i)w} h_t v_i + sum_{i<t} (t-1-i) e^{k_i-(t-1-i)w} h_t wkv_t,
  *   du =  sum_t h_t e^{u+k_t} v_t - sum_t h_t e^{u+k_t} wkv_t,
  * accumulated by the same recurrences run on |h_t|, |v_i|, |wkv_t|.
+ * dk_abs, dv_abs (B, T, C) (may be NULL) do the same for dk and dv, which are sums over
+ * the tokens t >= i that token i reaches:
+ *   dv_i = e^{k_i} h_i e^u + sum_{t>i} e^{k_i-(t-1-i)w} h_t,
+ *   dk_i = e^{k_i} h_i e^u v_i - e^{k_i} h_i e^u wkv_i
+ *        + sum_{t>i} e^{k_i-(t-1-i)w} h_t v_i - sum_{t>i} e^{k_i-(t-1-i)w} h_t wkv_t,
+ * so dv_abs_i = e^{k_i} (|h_i| e^u + sum |h_t| e^{-(t-1-i)w}) and dk_abs_i the same with
+ * (|v_i| + |wkv_t|) in each term: where the terms cancel, a float evaluation still
+ * rounds at their size.
  */
 int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const double *u,
                         const double *k, const double *v, const double *r, const double *dy,
                         double *dk, double *dv, double *dw, double *du, double *dr,
-                        double *dw_abs, double *du_abs)
+                        double *dw_abs, double *du_abs, double *dk_abs, double *dv_abs)
 {
     if (B < 0 || T < 0 || C < 0 || !w || !u || !k || !v || !dy || !dk || !dv || !dw || !du)
         return -1;
@@ -189,6 +197,10 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
                 double ek = exp(ki);
                 dv[AT(b, i, c)] = ek * (h * eu + beta);
                 dk[AT(b, i, c)] = ek * (h * eu * (vi - wkv[i]) + vi * beta - gamma);
+                if (dv_abs) dv_abs[AT(b, i, c)] = ek * (fabs(h) * eu + abeta);
+                if (dk_abs)
+                    dk_abs[AT(b, i, c)] = ek * (fabs(h) * eu * (fabs(vi) + fabs(wkv[i]))
+                                                + fabs(vi) * abeta + agamma);
                 dwc += -ek * (vi * betad - gammad);
                 duc += h * eu * ek * (vi - wkv[i]);
                 dwa += ek * (fabs(vi) * abetad + agammad);
@@ -234,9 +246,10 @@ int oracle_wkv_backward(int64_t B, int64_t T, int64_t C, const double *w, const 
  *   dr_t = dy_t wkv_t sigmoid(r_t) (1 - sigmoid(r_t)),
  * and finally dA0 = Abar_{-1}, dB0 = Bbar_{-1}.
  * A0, B0, gA, gB, dA0, dB0 are [B*C] and may be NULL (zero state / zero gradient / not
- * wanted). dw_abs, du_abs, dA0_abs, dB0_abs (may be NULL) receive the same sums run on
- * absolute values (|v|, |g|, |A0|, |gA|, |gB| in place of v, g, A0, gA, gB): the scale
- * against which a float evaluation of these sums is judged.
+ * wanted). dw_abs, du_abs, dA0_abs, dB0_abs, dk_abs, dv_abs (may be NULL) receive the
+ * same sums run on absolute values (|v|, |g|, |wkv|, |A0|, |gA|, |gB| in place of v, g,
+ * wkv, A0, gA, gB; dk_abs and dv_abs are (B, T, C) like dk and dv): the scale against
+ * which a float evaluation of these sums is judged.
  */
 int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
                               const double *u, const double *k, const double *v,
@@ -244,7 +257,8 @@ int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
                               const double *B0, const double *gA, const double *gB,
                               double *dk, double *dv, double *dw, double *du, double *dr,
                               double *dA0, double *dB0, double *dw_abs, double *du_abs,
-                              double *dA0_abs, double *dB0_abs)
+                              double *dA0_abs, double *dB0_abs, double *dk_abs,
+                              double *dv_abs)
 {
     if (B < 0 || T < 0 || C < 0 || !w || !u || !dw || !du) return -1;
     if (T > 0 && (!k || !v || !dy || !dk || !dv)) return -1;
@@ -293,6 +307,10 @@ int oracle_wkv_backward_state(int64_t B, int64_t T, int64_t C, const double *w,
                 /* Abar, Bbar here are dL/dA_t, dL/dB_t (this token's update feeds them) */
                 dv[AT(b, t, c)] = ek * Abar + g * bonus / D[t];
                 dk[AT(b, t, c)] = ek * (vt * Abar + Bbar) + g * bonus * (vt - wkv[t]) / D[t];
+                if (dv_abs) dv_abs[AT(b, t, c)] = ek * Abar_a + fabs(g) * bonus / D[t];
+                if (dk_abs)
+                    dk_abs[AT(b, t, c)] = ek * (fabs(vt) * Abar_a + Bbar_a)
+                                        + fabs(g) * bonus * (fabs(vt) + fabs(wkv[t])) / D[t];
                 dwc -= keep * (Aprev[t] * Abar + Bprev[t] * Bbar);
                 duc += g * bonus * (vt - wkv[t]) / D[t];
                 dwa += keep * (Aabs[t] * Abar_a + Bprev[t] * Bbar_a);

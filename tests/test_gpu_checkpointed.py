@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import wkv_inputs
-from wkv_check import assert_fp32_close
+from wkv_check import assert_fp32_close, assert_grad_close
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -67,8 +67,10 @@ def run(W, x, with_state=False, with_grad=False, gate=True, seed=0):
     assert W.wkv_stream_status() == 0
     ref = oracle.wkv_backward_state(x.w, x.u, x.k, x.v, x.r if gate else None, x.dy,
                                     A0, B0, gA, gB)
-    for n in ("dk", "dv") + (("dr",) if gate else ()):
-        assert_fp32_close(g[n].cpu().numpy(), ref[n], n)
+    for n in ("dk", "dv"):
+        assert_grad_close(g[n].cpu().numpy(), ref[n], ref[n + "_abs"], n)
+    if gate:
+        assert_fp32_close(g["dr"].cpu().numpy(), ref["dr"], "dr")
     for n in ("dw", "du"):
         assert_sum_close(g[n].cpu().numpy(), ref[n], ref[n + "_abs"], n)
     if with_state:

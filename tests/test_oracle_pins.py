@@ -336,6 +336,87 @@ def test_backward_state_chains_over_a_split_sequence():
     np.testing.assert_allclose(first["dB0"], whole["dB0"], rtol=1e-11, atol=1e-12)
 
 
+def _grad_terms_brute(w, u, k, v, r, dy, A0=None, B0=None, gA=None, gB=None):
+    """dk_abs, dv_abs by listing the terms of dk_i and dv_i one by one from the parallel
+    form (plain loops, tiny inputs): token i reaches output t >= i with the weight
+    e^{k_i - (t-1-i)w} / D_t (t > i) or e^{u+k_i} / D_t (t = i), and the final state with
+    e^{k_i - (T-1-i)w}; D_t, wkv_t are the definition's sums written out."""
+    B, T, C = k.shape
+    dka = np.zeros((B, T, C))
+    dva = np.zeros((B, T, C))
+    for b in range(B):
+        for c in range(C):
+            D = np.empty(T)
+            wkv = np.empty(T)
+            for t in range(T):
+                num = den = 0.0
+                if A0 is not None:
+                    num += math.exp(-t * w[c]) * A0[b, c]
+                    den += math.exp(-t * w[c]) * B0[b, c]
+                for i in range(t):
+                    e = math.exp(-(t - 1 - i) * w[c] + k[b, i, c])
+                    num += e * v[b, i, c]
+                    den += e
+                e = math.exp(u[c] + k[b, t, c])
+                D[t] = den + e
+                wkv[t] = (num + e * v[b, t, c]) / D[t]
+            g = dy[b, :, c] * (1.0 / (1.0 + np.exp(-r[b, :, c])) if r is not None else 1.0)
+            for i in range(T):
+                vi = abs(v[b, i, c])
+                e = math.exp(u[c] + k[b, i, c]) * abs(g[i]) / D[i]
+                sv, sk = e, e * (vi + abs(wkv[i]))
+                for t in range(i + 1, T):
+                    e = math.exp(k[b, i, c] - (t - 1 - i) * w[c]) * abs(g[t]) / D[t]
+                    sv += e
+                    sk += e * (vi + abs(wkv[t]))
+                if gA is not None:
+                    e = math.exp(k[b, i, c] - (T - 1 - i) * w[c])
+                    sv += e * abs(gA[b, c])
+                    sk += e * (vi * abs(gA[b, c]) + abs(gB[b, c]))
+                dva[b, i, c] = sv
+                dka[b, i, c] = sk
+    return dka, dva
+
+
+def test_gradient_term_scales_match_brute_force():
+    # dk_abs, dv_abs (the scale of the terms behind each dk, dv element) against the terms
+    # listed one by one, for the plain backward and through a state.
+    B, T, C = 2, 9, 3
+    w, u, k, v, r = _rand(B, T, C, 40, k_std=2.0)
+    g = np.random.Generator(np.random.PCG64(41))
+    dy = g.standard_normal((B, T, C))
+    a = oracle.wkv_backward(w, u, k, v, r, dy)
+    dka, dva = _grad_terms_brute(w, u, k, v, r, dy)
+    np.testing.assert_allclose(a["dk_abs"], dka, rtol=1e-12)
+    np.testing.assert_allclose(a["dv_abs"], dva, rtol=1e-12)
+    A0 = g.standard_normal((B, C))
+    B0 = g.uniform(0.5, 2.0, (B, C))
+    gA = g.standard_normal((B, C))
+    gB = g.standard_normal((B, C))
+    s = oracle.wkv_backward_state(w, u, k, v, r, dy, A0, B0, gA, gB)
+    dka, dva = _grad_terms_brute(w, u, k, v, r, dy, A0, B0, gA, gB)
+    np.testing.assert_allclose(s["dk_abs"], dka, rtol=1e-12)
+    np.testing.assert_allclose(s["dv_abs"], dva, rtol=1e-12)
+    for res in (a, s):
+        assert np.all(res["dv_abs"] >= np.abs(res["dv"]) * (1 - 1e-12))
+        assert np.all(res["dk_abs"] >= np.abs(res["dk"]) * (1 - 1e-12))
+
+
+def test_gradient_term_scales_without_cancellation():
+    # dy >= 0 and v >= 0 (hence wkv >= 0): every term of dv is non-negative, so
+    # dv_abs = dv; dk's terms are e^{..} h (v_i - wkv_t), so dk_abs = sum e^{..} h (v_i +
+    # wkv_t) = 2 v_i dv_i - dk_i.
+    B, T, C = 2, 50, 4
+    w, u, k, v, r = _rand(B, T, C, 42, k_std=2.0)
+    v = np.abs(v)
+    dy = np.abs(np.random.Generator(np.random.PCG64(43)).standard_normal((B, T, C)))
+    for res in (oracle.wkv_backward(w, u, k, v, r, dy),
+                oracle.wkv_backward_state(w, u, k, v, r, dy)):
+        np.testing.assert_allclose(res["dv_abs"], res["dv"], rtol=1e-12)
+        np.testing.assert_allclose(res["dk_abs"], 2 * v * res["dv"] - res["dk"], rtol=1e-10,
+                                   atol=1e-13)
+
+
 # ---- RWKV-7 generalised-delta-rule recurrence (research report, section 1.3.3) ----
 
 def _unit_rows(g, shape):

@@ -8,6 +8,11 @@ bf16 outputs:  |y - y_ref| <= ulp_bf16(y_ref) + 1e-5 * (1 + |y_ref|)
 States are compared through what the (a, b, p) representation leaves unique:
                rho = a / b and lambda = p + ln b, each within 1e-5 * (1 + |ref|).
 Reductions (dw, du) over n terms: |d - d_ref| <= 1e-5 * (1 + sum |terms|).
+Gradients dk, dv (each a sum over the later tokens a token reaches, plus the current
+               token's term): |d - d_ref| <= 1e-5 * (1 + sum |terms|) elementwise, with
+               sum |terms| the oracle's dk_abs, dv_abs. Where the terms do not cancel this
+               is the fp32 rule; where they do, a float evaluation rounds at the size of
+               the terms, not of their difference. dr (a product) keeps the fp32 rule.
 """
 import numpy as np
 
@@ -32,6 +37,23 @@ def assert_fp32_close(y, ref, what="y", tol=FP32_TOL):
             f"{what}: {int(bad.sum())} of {bad.size} elements outside 1e-5*(1+|ref|); worst at "
             f"{tuple(int(x) for x in i)}: got {np.asarray(y)[i]!r}, ref {np.asarray(ref)[i]!r}")
     return float((err / np.maximum(bound, 1e-300)).max()) if err.size else 0.0
+
+
+def assert_grad_close(got, ref, ref_abs, what, tol=FP32_TOL):
+    """dk / dv against the oracle, bounded by the size of their terms; returns the worst
+    error as a fraction of the bound."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.abs(got - ref)
+    bound = tol * (1.0 + np.asarray(ref_abs, dtype=np.float64))
+    bad = ~(err <= bound)
+    if bad.any():
+        i = np.unravel_index(np.argmax(np.where(bad, err / bound, 0)), err.shape)
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside 1e-5*(1+sum|terms|); "
+            f"worst at {tuple(int(x) for x in i)}: got {got[i]!r}, ref {ref[i]!r}, "
+            f"sum|terms| {float(np.asarray(ref_abs)[i])!r}")
+    return float((err / bound).max()) if err.size else 0.0
 
 
 def bf16_ulp(x):
