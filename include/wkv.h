@@ -124,10 +124,12 @@ WKV_API int wkv_forward_state(int64_t B, int64_t T, int64_t C, const float* w, c
  * memory, a deployment that forbids dynamic allocation after start-up).
  *
  * Same arguments, layout, semantics and results as wkv_forward_state; the caller passes
- * all inputs and outputs. The scratch of the chunked path (flags and published carries,
- * about 1 KiB per batch row x 32-channel group x 256-token segment) comes from a fixed
- * array of 8 MiB in the library's device memory, which every GPU that loads the library
- * holds until the process exits. Problems whose chunked
+ * all inputs and outputs. The scratch of the chunked path (a 4-byte flag and 1 KiB of
+ * published carries per item, an item being one batch row x 32-channel group x 256-token
+ * segment, plus a 16-byte header) comes from a fixed array of 8 MiB + 64 KiB in the
+ * library's device memory, which every GPU that loads the library holds until the process
+ * exits: up to 8223 items, e.g. one sequence of 32768 tokens x 2048 channels (8192
+ * items). The chunked path is taken below 8192 channels B*C. Problems whose chunked
  * plan needs more return WKV_ERR_SCRATCH_LIMIT before anything is enqueued; problems that
  * take the streaming path need no scratch and have no limit. Nothing is allocated: no
  * cudaMalloc, cudaMallocAsync or cudaFree (the flags are cleared with cudaMemsetAsync).

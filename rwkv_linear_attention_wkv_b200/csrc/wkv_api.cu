@@ -21,10 +21,14 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// The per-device cache is filled under a lock: host threads may make their first calls
+// on the same device at the same time.
 unsigned* error_word() {
   static unsigned* cached[kMaxDevices] = {};
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (cached[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;

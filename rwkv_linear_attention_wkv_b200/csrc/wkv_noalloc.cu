@@ -21,9 +21,12 @@ namespace wkv {
 
 namespace {
 
-// 8 MiB: the chunked path needs about 1 KiB per (batch row, 32-channel group, 256-token
-// segment), so this covers e.g. one sequence of 32768 tokens x 2048 channels.
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+// 8 MiB + 64 KiB. The chunked path needs 1 KiB of carries per item (batch row x
+// 32-channel group x 256-token segment) plus a 4-byte flag per item and a 16-byte ticket
+// header, so this holds up to 8223 items: e.g. one sequence of 32768 tokens x 2048
+// channels (8192 items, 8,421,392 bytes); one more segment (33024 tokens, 8256 items) is
+// over the limit.
+constexpr size_t kStaticScratchBytes = (size_t(8) << 20) + (size_t(64) << 10);
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
