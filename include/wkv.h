@@ -158,6 +158,28 @@ WKV_API int wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, con
                             float* b, float* p, cudaStream_t stream);
 
 /*
+ * S chained tokens for N sequences x L layers in one call, the state kept on chip between
+ * them (the news page "RWKV CUDA linear attention GPU", 技术深度解析, 持久化内核设计: a
+ * kernel that stays resident across token generations rather than one launch per token).
+ * Token s of every sequence and layer is the single-token step of wkv_decode_step applied
+ * to the state that token s - 1 left; the state is read once at the start and written
+ * once at the end, so a token moves 16 bytes per state (k, v, r in, y out) plus 24/S for
+ * the state, against 40 for separate wkv_decode_step calls. Results are bit for bit those
+ * of S wkv_decode_step calls.
+ *   k, v, r, y: fp32 [S, N, L, C] (token-major: token s is the [N, L, C] block at
+ *     s N L C); w, u: fp32 [L, C]; a, b, p: fp32 [N, L, C] state, read and updated in
+ *     place. r == NULL: no gate. y must not overlap k, v, r, a, b or p, and a, b, p must
+ *     not overlap each other or the inputs.
+ *   The tokens must be known in advance (as in prefill through a decode-shaped state
+ *   batch, or in checking several drafted tokens at once); a model whose next token
+ *   depends on this token's output calls wkv_decode_step per token.
+ * S == 0 or an empty batch: nothing is done. S >= 2^31: WKV_ERR_UNSUPPORTED.
+ */
+WKV_API int wkv_decode_steps(int64_t N, int64_t L, int64_t C, int64_t S, const float* w,
+                             const float* u, const float* k, const float* v, const float* r,
+                             float* y, float* a, float* b, float* p, cudaStream_t stream);
+
+/*
  * Backward of the forward (wkv_forward with the same w, u, k, v, r), fp32: gradients of
  * L = sum dy . y. The pages say only that the operator trains by ordinary backpropagation
  * (news page "RWKV CUDA linear attention GPU": fused forward and backward kernels); the

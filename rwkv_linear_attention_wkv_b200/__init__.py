@@ -12,6 +12,7 @@ import ctypes
 import os
 
 __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_step",
+           "wkv_decode_steps",
            "wkv_backward", "wkv_backward_state", "wkv_backward_workspace_bytes",
            "wkv_forward_checkpointed", "wkv_backward_checkpointed",
            "wkv7_forward", "wkv_stream_status", "wkv_status_string", "WkvError", "lib",
@@ -35,6 +36,7 @@ _SIGS = {
     "wkv_forward_bf16": ([_I, _I, _I] + [_P] * 6 + [_P], ctypes.c_int),
     "wkv_forward_state": ([_I, _I, _I] + [_P] * 12 + [_P], ctypes.c_int),
     "wkv_decode_step": ([_I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
+    "wkv_decode_steps": ([_I, _I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
     "wkv_stream_status": ([_P], ctypes.c_int),
     "wkv_backward_workspace_bytes": ([_I, _I, _I], ctypes.c_size_t),
     "wkv_backward": ([_I, _I, _I] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int),
@@ -188,6 +190,30 @@ def wkv_decode_step(w, u, k, v, r, a, b, p, y=None, stream=None):
     _need(y, "y", f32, (N, L, C))
     _call("wkv_decode_step", N, L, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
           _ptr(a), _ptr(b), _ptr(p), _stream(stream))
+    return y
+
+
+def wkv_decode_steps(w, u, k, v, r, a, b, p, y=None, stream=None):
+    """S chained tokens for [N, L, C] states in one call: k, v, r (S, N, L, C); w, u
+    [L, C]; (a, b, p) updated in place. Returns y (S, N, L, C)."""
+    torch = _torch()
+    if k.dim() != 4:
+        raise ValueError("k must be (S, N, L, C)")
+    S, N, L, C = k.shape
+    f32 = torch.float32
+    _need(k, "k", f32)
+    _need(v, "v", f32, (S, N, L, C))
+    if r is not None:
+        _need(r, "r", f32, (S, N, L, C))
+    for n, t in (("a", a), ("b", b), ("p", p)):
+        _need(t, n, f32, (N, L, C))
+    _need(w, "w", f32, (L, C))
+    _need(u, "u", f32, (L, C))
+    if y is None:
+        y = torch.empty((S, N, L, C), dtype=f32, device=k.device)
+    _need(y, "y", f32, (S, N, L, C))
+    _call("wkv_decode_steps", N, L, C, S, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r),
+          _ptr(y), _ptr(a), _ptr(b), _ptr(p), _stream(stream))
     return y
 
 

@@ -270,6 +270,22 @@ WKV_API int wkv_decode_step(int64_t N, int64_t L, int64_t C, const float* w, con
   return launch_decode(d, stream);
 }
 
+WKV_API int wkv_decode_steps(int64_t N, int64_t L, int64_t C, int64_t S, const float* w,
+                             const float* u, const float* k, const float* v, const float* r,
+                             float* y, float* a, float* b, float* p, cudaStream_t stream) {
+  if (N < 0 || L < 0 || C < 0 || S < 0) return WKV_ERR_INVALID_ARG;
+  if (N == 0 || L == 0 || C == 0 || S == 0) return WKV_OK;
+  if (!w || !u || !k || !v || !y || !a || !b || !p) return WKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {w, u, k, v, r, y, a, b, p};
+  for (const void* q : ptrs)
+    if (!aligned(q, 4)) return WKV_ERR_ALIGNMENT;
+  if (L > INT64_MAX / C || N > INT64_MAX / (L * C) || S >= (int64_t(1) << 31) ||
+      S > INT64_MAX / (N * L * C))
+    return WKV_ERR_UNSUPPORTED;
+  DecodeArgs d{N, L, C, w, u, k, v, r, y, a, b, p};
+  return launch_decode_steps(d, S, stream);
+}
+
 WKV_API size_t wkv_backward_workspace_bytes(int64_t B, int64_t T, int64_t C) {
   if (B <= 0 || T <= 0 || C <= 0) return 256;
   return backward_workspace_bytes(B, T, C);

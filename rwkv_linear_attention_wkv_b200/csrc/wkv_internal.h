@@ -70,6 +70,8 @@ struct DecodeArgs {
   float* p;
 };
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// S chained tokens: k, v, r, y are [S, N, L, C]; the state stays on chip between tokens.
+int launch_decode_steps(const DecodeArgs& a, int64_t S, cudaStream_t stream);
 
 // Backward over (B, T, C), fp32. r null: no gate (dr must be null). ws: device workspace of
 // backward_workspace_bytes(B, T, C) bytes, 256-byte aligned; no part needs clearing.
