@@ -12,8 +12,8 @@ Under torchrun (N > 1) every rank runs its own batch (seed = rank) with no colle
 the data path: weak scaling. Timing: CUDA events on the launching stream, barrier and
 synchronize on both sides, max over ranks. Rank 0 prints one JSON line.
 
---impl reference times the fp64 CPU oracle (single thread) on bounded samples of the
-same workload instead (rank 0 only).
+--impl reference times the fp64 CPU oracle on bounded samples of the same workload
+instead, on all of the host's cores (a process pool over channel blocks; rank 0 only).
 """
 from __future__ import annotations
 
@@ -35,6 +35,9 @@ UNIT = "G(B·T·C)/s"
 B, T, C = 8, 4096, 4096
 BYTES_PER_ELEM = 8          # read k, v, r and write y, 2 bytes each
 FALLBACK_HBM_GBS = 6650.0
+SPEC_HBM_GBS = 8000.0       # B200 HBM3e, nominal
+EXPS_PER_ELEM = 3           # two stabilised combines (ex2) and the gate's rcp: MUFU ops
+SUSTAINED_S = 1.2           # length of the sustained launch loop
 KERNEL = "wkv_fwd_tma_kernel<bf16, gate=1, TT=32, S=3, NW=1>"
 KERNEL_SOURCES = ["rwkv_linear_attention_wkv_b200/csrc/wkv_fwd.cu",
                   "rwkv_linear_attention_wkv_b200/csrc/wkv_window.cuh",
@@ -77,6 +80,86 @@ def hbm_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def peak_source():
+    """Where the HBM denominator comes from, for the JSON line."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return {"file": "MEASURED_PEAKS.json", "hbm_gbs": j.get("hbm_gbs"),
+                "how": j.get("how"), "when": j.get("when"), "gpu": j.get("gpu_name")}
+    except (OSError, ValueError):
+        return {"file": None, "hbm_gbs": FALLBACK_HBM_GBS,
+                "how": "fallback: an earlier copy measurement on this GPU type"}
+
+
+def sfu_peak(sm_max_mhz=None):
+    """MUFU operations per second from unit counts: 148 SMs x 16 per clock x the maximum
+    SM clock (a development probe of ex2.approx / rcp.approx measured 15.6 per clock per
+    SM, within 3% of it)."""
+    mhz = sm_max_mhz or 1965.0
+    return 148 * 16 * mhz * 1e6
+
+
+def host_cores():
+    """Cores this process may run on (what nproc reports)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _oracle_block(spec):
+    """Pool worker: the fp64 recurrence oracle, unchanged, on one block of channels of one
+    batch row, read from the memory-mapped inputs. Returns the elements computed."""
+    import numpy as np
+
+    import oracle
+    d, b, c0, c1 = spec
+    w = np.load(os.path.join(d, "w.npy"))[c0:c1]
+    u = np.load(os.path.join(d, "u.npy"))[c0:c1]
+    k, v, r = (np.ascontiguousarray(np.load(os.path.join(d, n + ".npy"),
+                                            mmap_mode="r")[b:b + 1, :, c0:c1])
+               for n in "kvr")
+    oracle.wkv_recurrent(w, u, k, v, r)
+    return k.size
+
+
+class OraclePool:
+    """The fp64 oracle on all host cores: a process pool (spawn start method, so nothing
+    is forked from a process that holds a CUDA context), each task one block of channels
+    of one batch row (channels are independent). The inputs go to .npy files in a
+    temporary directory that the workers map."""
+
+    def __init__(self, x, cores=None):
+        import concurrent.futures as cf
+        import multiprocessing as mp
+
+        import numpy as np
+        self.cores = cores or host_cores()
+        self.dir = tempfile.mkdtemp(prefix="wkv_oracle_")
+        for n in ("w", "u", "k", "v", "r"):
+            np.save(os.path.join(self.dir, n + ".npy"), getattr(x, n))
+        self.B, self.T, self.C = x.B, x.T, x.C
+        self.pool = cf.ProcessPoolExecutor(self.cores, mp_context=mp.get_context("spawn"))
+        # start every worker and load the oracle library before anything is timed
+        list(self.pool.map(_oracle_block, [(self.dir, 0, 0, 1)] * self.cores))
+
+    def run(self, b, c0, c1):
+        """Channels [c0, c1) of batch row b, split over the cores. Returns elements done."""
+        n = c1 - c0
+        pieces = max(1, min(n, 4 * self.cores))
+        cuts = [c0 + n * i // pieces for i in range(pieces + 1)]
+        specs = [(self.dir, b, cuts[i], cuts[i + 1]) for i in range(pieces)
+                 if cuts[i + 1] > cuts[i]]
+        return sum(self.pool.map(_oracle_block, specs))
+
+    def close(self):
+        import shutil
+        self.pool.shutdown()
+        shutil.rmtree(self.dir, ignore_errors=True)
 
 
 class ClockSampler:
@@ -139,6 +222,14 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def rank_batch(rank, Bn=B, Tn=T, Cn=C):
+    """The batch one rank works on: the 7B-shaped bf16 workload's distributions, seeded by
+    the rank, so every rank has its own independent batch (weak scaling, no collective on
+    the data path)."""
+    import wkv_inputs
+    return wkv_inputs.long_bf16(seed=rank, B=Bn, T=Tn, C=Cn)
+
+
 def max_over_ranks(values, dist=None, device="cpu"):
     """Element-wise maximum of a list of floats over all ranks (identity without dist)."""
     if dist is None:
@@ -165,55 +256,58 @@ def visible_gpu_indices(n):
     return list(range(n))
 
 
-def cpu_oracle_rate(x, budget_s=10.0, max_rows=None):
-    """fp64 recurrence oracle over whole batch rows of the workload until the budget is
-    spent (at least one row). Returns (elements per second, rows done)."""
-    import oracle
-    rows = 0
-    t0 = time.perf_counter()
-    nmax = x.B if max_rows is None else min(max_rows, x.B)
-    while rows < nmax:
-        oracle.wkv_recurrent(x.w, x.u, x.k[rows:rows + 1], x.v[rows:rows + 1],
-                             x.r[rows:rows + 1])
-        rows += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return rows * x.T * x.C / dt, rows
+def cpu_oracle_rate(x, budget_s=20.0):
+    """fp64 recurrence oracle over whole batch rows of the workload, on all host cores,
+    until the wall-clock budget is spent (at least one row). Returns (elements per second,
+    rows done, cores)."""
+    pool = OraclePool(x)
+    try:
+        rows = elems = 0
+        t0 = time.perf_counter()
+        while rows < x.B:
+            elems += pool.run(rows, 0, x.C)
+            rows += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+    finally:
+        pool.close()
+    return elems / dt, rows, pool.cores
 
 
 def run_reference(args, rank, world):
-    """The oracle as it stands, timed on this host's cores (one thread)."""
+    """The oracle as it stands, timed on all of this host's cores."""
     if rank != 0:
         return
     import numpy as np
 
-    import oracle
     import wkv_inputs
     x = wkv_inputs.long_bf16(seed=0, B=1)      # one batch row; steps sample channels of it
-    # Size each step so that warm-up + timed steps take about a minute in total.
-    probe_c = 64
-    t0 = time.perf_counter()
-    oracle.wkv_recurrent(x.w[:probe_c], x.u[:probe_c], x.k[:, :, :probe_c],
-                         x.v[:, :, :probe_c], x.r[:, :, :probe_c])
-    per_chan = (time.perf_counter() - t0) / probe_c
-    budget = 60.0 / max(1, args.steps + args.warmup)
-    nchan = int(max(8, min(x.C, budget / per_chan)))
-    g = np.random.Generator(np.random.PCG64(1))
-    times = []
-    for s in range(args.warmup + args.steps):
-        c0 = int(g.integers(0, x.C - nchan + 1))
-        sl = slice(c0, c0 + nchan)
-        k, v, r = (np.ascontiguousarray(a[:, :, sl]) for a in (x.k, x.v, x.r))
+    pool = OraclePool(x)
+    try:
+        # Size each step so that warm-up + timed steps take about a minute in total.
         t0 = time.perf_counter()
-        oracle.wkv_recurrent(x.w[sl], x.u[sl], k, v, r)
-        if s >= args.warmup:
-            times.append(time.perf_counter() - t0)
+        probe_c = 16 * pool.cores
+        pool.run(0, 0, probe_c)
+        per_chan = (time.perf_counter() - t0) / probe_c
+        budget = 60.0 / max(1, args.steps + args.warmup)
+        nchan = int(max(min(x.C, pool.cores), min(x.C, budget / per_chan)))
+        g = np.random.Generator(np.random.PCG64(1))
+        times = []
+        for s in range(args.warmup + args.steps):
+            c0 = int(g.integers(0, x.C - nchan + 1))
+            t0 = time.perf_counter()
+            pool.run(0, c0, c0 + nchan)
+            if s >= args.warmup:
+                times.append(time.perf_counter() - t0)
+    finally:
+        pool.close()
     elems = nchan * x.T
     total = sum(times)
     value = elems * len(times) / total / 1e9
     sample = (f"per step {nchan} channels x {x.T} tokens of batch row 0 of the B=8,T=4096,"
-              f"C=4096 bf16 workload; fp64 recurrence, 1 thread")
+              f"C=4096 bf16 workload; fp64 recurrence on {pool.cores} host cores (process pool "
+              "over channel blocks)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -221,7 +315,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "WKV forward, B=8 T=4096 C=4096 (oracle on a sample)",
                    "B": B, "T": T, "C": C, "sample": sample},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": pool.cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -244,7 +338,7 @@ def run_ours(args, rank, world, local_rank):
 
     Bn, Tn = args.batch, args.seq or T
     ELEMS = Bn * Tn * C
-    x = wkv_inputs.long_bf16(seed=rank, B=Bn, T=Tn)
+    x = rank_batch(rank, Bn, Tn)
 
     def to_bf16(bits, pin=False):
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
@@ -285,6 +379,27 @@ def run_ours(args, rank, world, local_rank):
     elapsed_ms, launch_ms = max_over_ranks(
         [starts[0].elapsed_time(ends[-1]), statistics.mean(per_launch)], dist, dev)
     value = aggregate_rate(world, ELEMS, args.steps, elapsed_ms)
+
+    # Sustained: back-to-back launches for at least SUSTAINED_S seconds (the power cap and
+    # the clock it settles at show over such a loop, not over a short burst), with its
+    # own clock record.
+    n_sus = max(args.steps, int(SUSTAINED_S / (launch_ms / 1e3)) + 1)
+    sus_sampler = ClockSampler(visible_gpu_indices(world) if rank == 0 else None)
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    if rank == 0:
+        sus_sampler.__enter__()
+    s0.record(stream)
+    for _ in range(n_sus):
+        W.wkv_forward_bf16(w, u, k, v, r, y=y)
+    s1.record(stream)
+    barrier()
+    if rank == 0:
+        sus_sampler.__exit__(None, None, None)
+    if W.wkv_stream_status() != 0:
+        raise RuntimeError("device-side error during the sustained loop")
+    (sus_ms,) = max_over_ranks([s0.elapsed_time(s1)], dist, dev)
 
     # End to end through the public API: pinned host k, v, r -> device, forward, y -> host,
     # every step. Steps are pipelined over two device buffer sets and three streams (copy
@@ -350,31 +465,58 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return
     peak, peak_kind = hbm_peak()
-    achieved = ELEMS * BYTES_PER_ELEM / (launch_ms / 1e3) / 1e9
+    clocks = sampler.summary()
+    sus_clocks = sus_sampler.summary()
+    algo_bytes = ELEMS * BYTES_PER_ELEM
+    achieved = algo_bytes / (launch_ms / 1e3) / 1e9
+    # Roofline: max(bytes / HBM peak, MUFU operations / MUFU peak) against the mean launch.
+    exps = EXPS_PER_ELEM * ELEMS
+    sfu = sfu_peak(clocks.get("sm_max_mhz"))
+    t_hbm_ms = algo_bytes / (peak * 1e9) * 1e3
+    t_sfu_ms = exps / sfu * 1e3
+    traffic = measured_traffic()
+    sus_launch_ms = sus_ms / n_sus
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rate, rows = cpu_oracle_rate(x, budget_s=10.0)
-        cpu = {"value": rate / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        rate, rows, cores = cpu_oracle_rate(x, budget_s=20.0)
+        cpu = {"value": rate / 1e9, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{rows} of {Bn} batch rows ({rows} x {Tn} x 4096 elements) of the "
-                         f"same inputs, fp64 recurrence, 1 thread"}
-    clocks = sampler.summary()
+                         f"same inputs, fp64 recurrence, process pool over channel blocks on "
+                         f"{cores} host cores"}
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
+        "storage_dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"WKV forward bf16 in/out, B={Bn} T={Tn} C=4096 (7B-shaped, "
                                "k spikes of +60), one batch per GPU",
-                   "B": Bn, "T": Tn, "C": C, "storage": "bf16", "global_batch": Bn * world,
+                   "B": Bn, "T": Tn, "C": C, "storage": "bf16 k, v, r, y",
+                   "arithmetic": "fp32 (w, u fp32)", "global_batch": Bn * world,
                    "seq_len": Tn, "parallelism": f"dp{world} (independent batches)",
                    "l2": f"inputs {3 * ELEMS * 2 / 1e6:.0f} MB + output {ELEMS * 2 / 1e6:.0f} MB "
                          "per step > 126 MB L2; no flush",
                    "kernel": KERNEL},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": measured_traffic(),
-                     "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": ELEMS * BYTES_PER_ELEM,
+        "roofline": {"bound": "hbm" if t_hbm_ms >= t_sfu_ms else "sfu",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": max(t_hbm_ms, t_sfu_ms) / launch_ms,
+                     "traffic": traffic,
+                     "traffic_source": ("ncu dram__bytes_read.sum + dram__bytes_write.sum "
+                                        f"from {TRAFFIC_FILE} (taken on these kernel sources)"
+                                        if traffic is not None else None),
+                     "peak_kind": peak_kind, "peak_source": peak_source(),
+                     "frac_of_spec_8TBs": achieved / SPEC_HBM_GBS,
+                     "algorithmic_bytes_per_launch": algo_bytes,
+                     "hbm_time_ms": t_hbm_ms, "hbm_frac": t_hbm_ms / launch_ms,
+                     "exps": exps, "sfu_peak_per_s": sfu,
+                     "sfu_peak_kind": "unit counts: 148 SMs x 16 MUFU/clk x max SM clock",
+                     "sfu_time_ms": t_sfu_ms, "sfu_frac": t_sfu_ms / launch_ms,
                      "launch_ms": launch_ms},
+        "sustained": {"launches": n_sus, "seconds": sus_ms / 1e3,
+                      "ms_per_launch": sus_launch_ms,
+                      "value": aggregate_rate(world, ELEMS, n_sus, sus_ms),
+                      "achieved_GBps": algo_bytes / (sus_launch_ms / 1e3) / 1e9,
+                      "frac": algo_bytes / (sus_launch_ms / 1e3) / 1e9 / peak,
+                      "clocks": sus_clocks},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": 3 * ELEMS * 2, "d2h_bytes_per_step": ELEMS * 2,
@@ -503,6 +645,24 @@ def run_workload(args):
                         args.warmup, stream)
         line("decode", "decode step fp32 256 seq x 32 layers x 4096 (state in place)", ms, n,
              40 * n, {"tokens_per_s": dd.N / (ms / 1e3)})
+        # S tokens per call with the state kept on chip (wkv_decode_steps): per token
+        # 16 bytes per state (k, v, r in, y out) plus the state once per call (24 / S).
+        S = 64
+        ks = torch.empty((S,) + tuple(k.shape), device=dev)
+        vs, rs = torch.empty_like(ks), torch.empty_like(ks)
+        for s_ in range(S):
+            kk, vv, rr = dd.step(s_)
+            ks[s_].copy_(torch.from_numpy(kk))
+            vs[s_].copy_(torch.from_numpy(vv))
+            rs[s_].copy_(torch.from_numpy(rr))
+        ys = torch.empty_like(ks)
+        steps = max(3, args.steps // S)
+        ms = _time_loop(lambda: W.wkv_decode_steps(w, u, ks, vs, rs, a, b, p, y=ys), steps,
+                        3, stream)
+        line("decode", f"decode_steps fp32 256 seq x 32 layers x 4096, {S} tokens per call "
+             "(state on chip between tokens); ms and rates per token", ms / S, n,
+             int(16 * n + 24 * n / S), {"tokens_per_s": dd.N * S / (ms / 1e3),
+                                        "ms_per_call": ms, "tokens_per_call": S})
     elif args.workload == "rwkv7":
         T7 = args.seq or 4096
         x = wkv_inputs.rwkv7_inputs(8, T7, 64, seed=0)
@@ -531,7 +691,7 @@ def run_workload(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
