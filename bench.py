@@ -682,6 +682,32 @@ def run_workload(args):
              {"flops": flops, "achieved_TFLOPs": flops / (ms / 1e3) / 1e12,
               "alu_peak_TFLOPs": alu_peak / 1e12,
               "alu_frac": flops / (ms / 1e3) / alu_peak})
+    elif args.workload == "mstate":
+        # Matrix-valued state without the delta term: the chunked tensor-core kernel and the
+        # token-by-token recurrence kernel on the same inputs (a = b = 0).
+        T7 = args.seq or 4096
+        x = wkv_inputs.rwkv7_inputs(8, T7, 64, seed=0)
+        x.a[...] = 0.0
+        x.b[...] = 0.0
+        t = {nm: d(getattr(x, nm)) for nm in ("r", "w", "k", "v", "a", "b")}
+        s0 = d(x.S0)
+        y = torch.empty_like(t["k"])
+        s1 = torch.empty_like(s0)
+        n = x.B * x.T * x.H * x.N
+        # per token and head: A (N L), A V (N L / 2 on average), R~ S0^T (N^2), V^T K~
+        # (N^2) multiply-adds with L = N = 64 as 3 tf32 products each
+        tc_flops = 3 * 2 * (64 * 64 + 64 * 32 + 64 * 64 + 64 * 64) * x.B * x.T * x.H
+        ms = _time_loop(lambda: W.wkv_mstate_forward(*(t[nm] for nm in "rwkv"), state=s0, y=y,
+                                                     state_out=s1), args.steps, args.warmup,
+                        stream)
+        line("mstate", f"matrix-state WKV fp32 8x{x.T}x64 heads x 64, chunked on tcgen05 "
+             "(3 x tf32 products)", ms, n, 20 * n + 8 * x.B * x.H * x.N * x.N,
+             {"tf32_flops_issued": tc_flops,
+              "tf32_TFLOPs": tc_flops / (ms / 1e3) / 1e12})
+        ms = _time_loop(lambda: W.wkv7_forward(*(t[nm] for nm in "rwkvab"), state=s0, y=y,
+                                               state_out=s1), args.steps, args.warmup, stream)
+        line("mstate", f"same inputs through the recurrence kernel (wkv7_forward, a = b = 0)",
+             ms, n, 28 * n + 8 * x.B * x.H * x.N * x.N)
     else:
         raise SystemExit(f"unknown workload {args.workload}")
     if W.wkv_stream_status() != 0:
@@ -699,7 +725,7 @@ def main():
                     help="batch rows per GPU (default 8, the measured workload; smaller "
                          "values are for profiler captures)")
     ap.add_argument("--workload", default="bf16_7b",
-                    choices=["bf16_7b", "train_169m", "long_ctx", "decode", "rwkv7"],
+                    choices=["bf16_7b", "train_169m", "long_ctx", "decode", "rwkv7", "mstate"],
                     help="bf16_7b (default) prints the benchmark line; the others print "
                          "measurements of the other workloads, one GPU")
     ap.add_argument("--seq", type=int, default=None,

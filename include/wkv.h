@@ -64,8 +64,11 @@ typedef enum wkv_status {
   WKV_ERR_UNSUPPORTED = 5, /* a size beyond what the kernels index (e.g. T >= 2^31), or
                               a shape an entry point's kernels cannot take (documented
                               with the entry point)                                       */
-  WKV_ERR_SCRATCH_LIMIT = 6 /* wkv_forward_state_static: the problem needs more scratch
-                               than the library's fixed array holds                       */
+  WKV_ERR_SCRATCH_LIMIT = 6, /* wkv_forward_state_static: the problem needs more scratch
+                                than the library's fixed array holds                      */
+  WKV_ERR_RANGE = 7          /* reported by wkv_stream_status: an input lay outside the
+                                range a kernel handles (wkv_mstate_forward: a decay too
+                                strong within a chunk); the outputs are then undefined     */
 } wkv_status;
 
 /* Human-readable name of a status code. Never NULL. */
@@ -285,10 +288,39 @@ WKV_API int wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float
                          cudaStream_t stream);
 
 /*
+ * Matrix-valued-state WKV with a per-key-channel, data-dependent decay, fp32: the RWKV-5/6
+ * form (research report "RWKV模型深度研究报告", section 1.3.2: a matrix-valued state per
+ * head, each feature channel with its own time decay), computed chunkwise with matrix
+ * products inside each chunk of 64 tokens and the state carried between chunks (section
+ * 1.4.1), the products on the tensor cores. Per head of N channels:
+ *   S_t[i][j] = S_{t-1}[i][j] w_t[j] + v_t[i] k_t[j],    y_t[i] = sum_j S_t[i][j] r_t[j]
+ * i.e. wkv7_forward with a = b = 0 (section 1.3.3's update without the delta term), and
+ * the same read-out and layouts:
+ *   r, w, k, v, y: fp32 (B, T, H, N) row-major; w the decay factor itself (in (0, 1]).
+ *   s0: initial state (B, H, N, N), S[i][j] at i N + j; NULL = zero. s1: final state, same
+ *     layout; NULL = not wanted; may alias s0.
+ * Numerics: the products run as three tf32 tensor-core products of operands split into
+ * tf32 high and low parts, accumulated in fp32 (about 2^-22 relative error per product).
+ * Range: the decay over any 31 or 32 consecutive tokens aligned to half a chunk must stay
+ * above 2^-60 per channel (e.g. w >= 0.27 on every token); otherwise wkv_stream_status()
+ * reports WKV_ERR_RANGE and y, s1 are undefined (wkv7_forward with a = b = 0 handles any
+ * decay, token by token).
+ * N must be 64 (else WKV_ERR_UNSUPPORTED); every pointer 16-byte aligned (else
+ * WKV_ERR_ALIGNMENT); y must not overlap the inputs or the states. T == 0: s1 = s0 (zero
+ * if s0 is NULL). Scratch (a two-slot state ring per head, 32 KiB per (batch row, head))
+ * is allocated with cudaMallocAsync on `stream` and freed in stream order. Chunks of one
+ * head wait for one another on the device, with bounded waits (WKV_ERR_TIMEOUT).
+ */
+WKV_API int wkv_mstate_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float* r,
+                               const float* w, const float* k, const float* v, float* y,
+                               const float* s0, float* s1, cudaStream_t stream);
+
+/*
  * Query and clear device-side errors. Synchronises `stream`, then returns WKV_ERR_TIMEOUT
  * if any kernel of this library on the current device gave up a bounded wait since the
- * last query (the outputs of that call are then undefined), WKV_ERR_CUDA if the stream
- * reports a CUDA error, else WKV_OK.
+ * last query, else WKV_ERR_RANGE if a kernel met an input outside its range (the outputs
+ * of that call are undefined in both cases), WKV_ERR_CUDA if the stream reports a CUDA
+ * error, else WKV_OK.
  */
 WKV_API int wkv_stream_status(cudaStream_t stream);
 

@@ -15,7 +15,7 @@ __all__ = ["wkv_forward", "wkv_forward_bf16", "wkv_forward_state", "wkv_decode_s
            "wkv_decode_steps",
            "wkv_backward", "wkv_backward_state", "wkv_backward_workspace_bytes",
            "wkv_forward_checkpointed", "wkv_backward_checkpointed",
-           "wkv7_forward", "wkv_stream_status", "wkv_status_string", "WkvError", "lib",
+           "wkv7_forward", "wkv_mstate_forward", "wkv_stream_status", "wkv_status_string", "WkvError", "lib",
            "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwkv.so")
@@ -44,6 +44,7 @@ _SIGS = {
                                    ctypes.c_int),
     "wkv_backward_state": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int),
     "wkv7_forward": ([_I, _I, _I, _I] + [_P] * 9 + [_P], ctypes.c_int),
+    "wkv_mstate_forward": ([_I, _I, _I, _I] + [_P] * 7 + [_P], ctypes.c_int),
     "wkv_forward_checkpointed": ([_I, _I, _I] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int),
     "wkv_backward_checkpointed": ([_I, _I, _I] + [_P] * 21 + [ctypes.c_size_t, _P],
                                   ctypes.c_int),
@@ -390,6 +391,33 @@ def wkv7_forward(r, w, k, v, a, b, state=None, y=None, state_out=None, want_stat
         _need(s1, "state_out", f32, (B, H, N, N))
     _call("wkv7_forward", B, T, H, N, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
           _ptr(y), _ptr(state), _ptr(s1), _stream(stream))
+    return y, s1
+
+
+def wkv_mstate_forward(r, w, k, v, state=None, y=None, state_out=None, want_state=True,
+                       stream=None):
+    """Matrix-valued-state WKV (per-key-channel decay, no delta term), chunked on the tensor
+    cores: r, w, k, v fp32 (B, T, H, N), N = 64; state (B, H, N, N) or None (zero). Returns
+    (y, S_T), or (y, None) with want_state=False. state_out may be `state` itself."""
+    torch = _torch()
+    f32 = torch.float32
+    if k.dim() != 4:
+        raise ValueError("k must be (B, T, H, N)")
+    B, T, H, N = k.shape
+    for n, t in (("r", r), ("w", w), ("k", k), ("v", v)):
+        _need(t, n, f32, (B, T, H, N))
+    if y is None:
+        y = torch.empty((B, T, H, N), dtype=f32, device=k.device)
+    _need(y, "y", f32, (B, T, H, N))
+    if state is not None:
+        _need(state, "state", f32, (B, H, N, N))
+    s1 = None
+    if want_state:
+        s1 = state_out if state_out is not None else torch.empty((B, H, N, N), dtype=f32,
+                                                                 device=k.device)
+        _need(s1, "state_out", f32, (B, H, N, N))
+    _call("wkv_mstate_forward", B, T, H, N, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(y),
+          _ptr(state), _ptr(s1), _stream(stream))
     return y, s1
 
 

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "wkv_device.cuh"
 #include "wkv_internal.h"
 #include "wkv_testing.h"
 
@@ -229,6 +230,7 @@ WKV_API const char* wkv_status_string(int status) {
     case WKV_ERR_TIMEOUT: return "WKV_ERR_TIMEOUT";
     case WKV_ERR_UNSUPPORTED: return "WKV_ERR_UNSUPPORTED";
     case WKV_ERR_SCRATCH_LIMIT: return "WKV_ERR_SCRATCH_LIMIT";
+    case WKV_ERR_RANGE: return "WKV_ERR_RANGE";
     default: return "WKV_ERR_UNKNOWN";
   }
 }
@@ -363,6 +365,36 @@ WKV_API int wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float
   return launch_wkv7(B, T, H, r, w, k, v, a, b, y, s0, s1, err, stream);
 }
 
+WKV_API int wkv_mstate_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float* r,
+                               const float* w, const float* k, const float* v, float* y,
+                               const float* s0, float* s1, cudaStream_t stream) {
+  if (B < 0 || T < 0 || H < 0 || N < 0) return WKV_ERR_INVALID_ARG;
+  if (B == 0 || H == 0) return WKV_OK;
+  if (N != 64) return WKV_ERR_UNSUPPORTED;
+  if (T > 0 && (!r || !w || !k || !v || !y)) return WKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {r, w, k, v, y, s0, s1};
+  for (const void* q : ptrs)
+    if (!aligned(q, 16)) return WKV_ERR_ALIGNMENT;
+  if (T >= (int64_t(1) << 31) || B * H >= (int64_t(1) << 24) ||
+      (T > 0 && B > INT64_MAX / T / (H * N)) || B * H * ((T + 63) / 64) >= (int64_t(1) << 31))
+    return WKV_ERR_UNSUPPORTED;
+  const size_t sbytes = size_t(B) * H * N * N * sizeof(float);
+  if (T == 0) {  // no tokens: the state passes through
+    if (s1 == nullptr || s1 == s0) return WKV_OK;
+    const cudaError_t e = s0 ? cudaMemcpyAsync(s1, s0, sbytes, cudaMemcpyDeviceToDevice, stream)
+                             : cudaMemsetAsync(s1, 0, sbytes, stream);
+    return e == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+  }
+  unsigned* err = error_word();
+  if (err == nullptr) return WKV_ERR_CUDA;
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, mstate_scratch_bytes(B, H), stream) != cudaSuccess)
+    return WKV_ERR_CUDA;
+  const int rc = launch_mstate(B, T, H, r, w, k, v, y, s0, s1, ws, err, stream);
+  cudaFreeAsync(ws, stream);
+  return rc;
+}
+
 WKV_API int wkv_stream_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return WKV_ERR_CUDA;
   unsigned* err = error_word();
@@ -371,7 +403,7 @@ WKV_API int wkv_stream_status(cudaStream_t stream) {
   if (cudaMemcpy(&h, err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return WKV_ERR_CUDA;
   if (h != 0) {
     if (cudaMemset(err, 0, sizeof(unsigned)) != cudaSuccess) return WKV_ERR_CUDA;
-    return WKV_ERR_TIMEOUT;
+    return (h & kErrTimeout) ? WKV_ERR_TIMEOUT : WKV_ERR_RANGE;
   }
   return WKV_OK;
 }

@@ -20,6 +20,7 @@ constexpr float kEmptyLogScale = -1.0e38f;
 
 // Error word bits, written by kernels and read back by wkv_stream_status().
 constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrRange = 2u;   // an input outside the range a kernel handles
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -174,6 +175,11 @@ __device__ __forceinline__ void tma_store_wait_all() {
 // Generic-proxy writes to shared memory become visible to the async proxy (TMA store).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Bring the 128-byte line at p into L2 (no register result, nothing waits for it).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {

@@ -73,6 +73,13 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // S chained tokens: k, v, r, y are [S, N, L, C]; the state stays on chip between tokens.
 int launch_decode_steps(const DecodeArgs& a, int64_t S, cudaStream_t stream);
 
+// Matrix-valued-state forward (heads of 64), chunked on the tensor cores. scratch: device
+// memory of mstate_scratch_bytes(B, H) bytes (cleared in part by the launcher).
+size_t mstate_scratch_bytes(int64_t B, int64_t H);
+int launch_mstate(int64_t B, int64_t T, int64_t H, const float* r, const float* w,
+                  const float* k, const float* v, float* y, const float* s0, float* s1,
+                  void* scratch, unsigned* err, cudaStream_t stream);
+
 // Backward over (B, T, C), fp32. r null: no gate (dr must be null). ws: device workspace of
 // backward_workspace_bytes(B, T, C) bytes, 256-byte aligned; no part needs clearing.
 struct BwdArgs {
