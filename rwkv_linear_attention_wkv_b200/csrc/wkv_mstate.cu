@@ -38,8 +38,8 @@
 // 1024). An operand is three such tiles (hi, mid, lo: 24 KiB). Every operand is K-major
 // (in this layout MN-major tf32 operands read as zeros, measured): R~ and K~ token-major,
 // K~ also transposed (rows = key channel j), V transposed (rows = value channel i). After
-// the first products the K~ tiles take (S_0 o gamma_m), and after the second the R~
-// tiles take A.
+// the first products (D_A, D_U) the K~ tiles take (S_0 o gamma_m) and the K~^T tiles take A,
+// so that the inter-chunk term and A V run together as the second and last MMA phase.
 // Tensor memory: 256 columns, each result a (main, correction) pair of 64-column
 // accumulators (M = 64 layout): D_A at 0/64, D_U (= V^T K~) at 128/192, and D_Y at 128/192
 // once D_U has been read.
@@ -58,8 +58,8 @@ constexpr uint32_t kTile = 8192;        // bytes of a 64 x 64 bf16 tile
 constexpr uint32_t kOp = 3 * kTile;     // an operand: hi, mid, lo tiles
 constexpr int kGP = 68;                 // row pitch (floats) of the decay table
 constexpr uint32_t kOffR = 0, kOffK = kOp, kOffKt = 2 * kOp, kOffV = 3 * kOp;  // G in V's space
-constexpr uint32_t kOffVec = 4 * kOp;                      // gref, g63 [64] each
-constexpr uint32_t kSmemBytes = kOffVec + 2 * kHN * 4;
+constexpr uint32_t kOffVec = 4 * kOp;  // gref, g63 [64] each, quarter totals [4][64]
+constexpr uint32_t kSmemBytes = kOffVec + 6 * kHN * 4;
 constexpr uint32_t kTmemCols = 256;
 static_assert(kCL * kGP * 4 <= kOp, "the decay table must fit in V's space");
 
@@ -95,31 +95,34 @@ __device__ __forceinline__ void st_row4(unsigned char* op, int row, int col, con
   for (int t = 0; t < 3; ++t) *reinterpret_cast<uint2*>(op + t * kTile + off) = s.p[t];
 }
 
-// Elements (row .. row + 3, col) of an operand's three tiles: the transpose of st_row4.
+// Elements (row .. row + 3, col), row % 4 == 0, of an operand's three tiles: the transpose
+// of st_row4. The four rows share a core matrix, 16 bytes apart.
 __device__ __forceinline__ void st_col4(unsigned char* op, int row, int col, const Split4& s) {
+  unsigned char* const at = op + el_off(row, col);
 #pragma unroll
   for (int t = 0; t < 3; ++t) {
     const uint32_t lo = s.p[t].x, hi = s.p[t].y;
-    unsigned char* tile = op + t * kTile;
-    *reinterpret_cast<uint16_t*>(tile + el_off(row + 0, col)) = uint16_t(lo);
-    *reinterpret_cast<uint16_t*>(tile + el_off(row + 1, col)) = uint16_t(lo >> 16);
-    *reinterpret_cast<uint16_t*>(tile + el_off(row + 2, col)) = uint16_t(hi);
-    *reinterpret_cast<uint16_t*>(tile + el_off(row + 3, col)) = uint16_t(hi >> 16);
+    *reinterpret_cast<uint16_t*>(at + t * kTile + 0) = uint16_t(lo);
+    *reinterpret_cast<uint16_t*>(at + t * kTile + 16) = uint16_t(lo >> 16);
+    *reinterpret_cast<uint16_t*>(at + t * kTile + 32) = uint16_t(hi);
+    *reinterpret_cast<uint16_t*>(at + t * kTile + 48) = uint16_t(hi >> 16);
   }
 }
 
-// The 64 x 64 x 64 product of two split operands (A: rows M, cols K; B: rows N, cols K):
+// The 64 x 64 x 64 product of two split operands (A: rows M, cols K; B: rows N, cols K),
+// given the descriptors of their hi tiles (an operand's tiles and K steps differ only in
+// the start-address field, so each MMA's descriptor is the base plus a constant):
 // hi.hi into d, the five correction products into d + 64. accumulate: add to d, d + 64.
-__device__ __forceinline__ void mma_split(uint32_t d, uint32_t a, uint32_t b, bool accumulate) {
+__device__ __forceinline__ void mma_split(uint32_t d, uint64_t a, uint64_t b, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16(64, 64);
   // (a part, b part) in tiles: hi = 0, mid = 1, lo = 2
-  const int pa[6] = {0, 0, 1, 0, 2, 1}, pb[6] = {0, 1, 0, 2, 0, 1};
+  constexpr int pa[6] = {0, 0, 1, 0, 2, 1}, pb[6] = {0, 1, 0, 2, 0, 1};
 #pragma unroll
   for (int p = 0; p < 6; ++p)
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks)
-      mma_bf16(p == 0 ? d : d + 64, smem_desc(a + pa[p] * kTile + ks * 256, 128, 1024),
-               smem_desc(b + pb[p] * kTile + ks * 256, 128, 1024), idesc,
+      mma_bf16(p == 0 ? d : d + 64, a + uint64_t((pa[p] * kTile + ks * 256) >> 4),
+               b + uint64_t((pb[p] * kTile + ks * 256) >> 4), idesc,
                (accumulate || ks > 0 || p > 1) ? 1u : 0u);
 }
 
@@ -131,6 +134,18 @@ __device__ __forceinline__ void tmem_ld16_pair(uint32_t taddr, float (&v)[16]) {
   tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __fadd_rn(v[i], c[i]);
+}
+
+// An M = 64 result fills lanes 0-15 of each sub-partition, so after a 16-column load only
+// lanes 0-15 hold data. Hand the upper 8 of those 16 columns to lanes 16-31 (lane l + 16
+// takes lane l's), so that each lane works on 8 columns of row (lane % 16): columns
+// 0-7 of the 16 in lanes 0-15, 8-15 in lanes 16-31.
+__device__ __forceinline__ void half_row(const float (&v)[16], float (&x)[8], int lane) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float up = __shfl_sync(0xffffffffu, v[8 + i], lane & 15);
+    x[i] = lane < 16 ? v[i] : up;
+  }
 }
 
 constexpr int kThreads = 256;
@@ -151,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
   float* const G = reinterpret_cast<float*>(smem + kOffV);  // [64][kGP], until V is split
   float* const gref = reinterpret_cast<float*>(smem + kOffVec);
   float* const g63 = gref + kHN;
+  float* const qtot = g63 + kHN;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = B * H;
@@ -169,6 +185,9 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = tmem_slot;
+  const uint32_t sb = smem_u32(smem);
+  const uint64_t aR = smem_desc(sb + kOffR, 128, 1024), aK = smem_desc(sb + kOffK, 128, 1024),
+                 aKt = smem_desc(sb + kOffKt, 128, 1024), aV = smem_desc(sb + kOffV, 128, 1024);
   unsigned item = s_item;
   uint32_t phase = 0;  // parity of the next completion of the MMA barrier
 
@@ -231,30 +250,41 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
     }
   }
 
-  // Decays of the chunk, per key channel j, in two halves of 32 tokens (thread (j, half)):
-  // the first half's running product gamma_t ends at gamma_m (m = 31) and gives
-  // G_t = gamma_t / gamma_m; the second half's running product from token 32 is G_t itself.
-  if (tid < 128) {
-    const int j = tid & 63, half = tid >> 6;
-    float p[32];
+  // Decays of the chunk, per key channel j, in quarters of 16 tokens (thread (j, q)): a
+  // running product p_t within each quarter and the quarter totals Q_0..Q_3; then
+  // gamma_t = Q_0 p_t (second quarter), gamma_m = Q_0 Q_1 (m = 31), and G_t = gamma_t /
+  // gamma_m in the first half, G_t = p_t (third quarter) or Q_2 p_t (fourth) in the second.
+  {
+    const int j = tid & 63, qtr = tid >> 6;
+    float p[16];
 #pragma unroll
-    for (int t = 0; t < 32; ++t) p[t] = G[(32 * half + t) * kGP + j];
+    for (int t = 0; t < 16; ++t) p[t] = G[(16 * qtr + t) * kGP + j];
 #pragma unroll
-    for (int t = 1; t < 32; ++t) p[t] = __fmul_rn(p[t - 1], p[t]);
-    if (half == 0) {
-      const float gm = p[31];
+    for (int t = 1; t < 16; ++t) p[t] = __fmul_rn(p[t - 1], p[t]);
+    qtot[qtr * kHN + j] = p[15];
+    __syncthreads();
+    const float q0 = qtot[j], q1 = qtot[kHN + j], q2 = qtot[2 * kHN + j];
+    if (qtr < 2) {
+      const float gm = __fmul_rn(q0, q1);
+      const float f = __fmul_rn(qtr == 1 ? q0 : 1.f, __frcp_rn(gm));
 #pragma unroll
-      for (int t = 0; t < 32; ++t) G[t * kGP + j] = __fdiv_rn(p[t], gm);
-      gref[j] = gm;
-      // The factorisation needs the decay over each half of the chunk to stay above 2^-60
-      // (G_0 = 1 / (w_1 ... w_31), G_63 = w_32 ... w_63); beyond that R~ or K~ could leave
-      // the float range. Flag it rather than return infinities silently.
-      if (!(G[j] <= 0x1p60f)) atomicOr(err, kErrRange);
+      for (int t = 0; t < 16; ++t) G[(16 * qtr + t) * kGP + j] = __fmul_rn(f, p[t]);
+      if (qtr == 0) {
+        gref[j] = gm;
+        // The factorisation needs the decay over each half of the chunk to stay above
+        // 2^-60 (G_0 = 1 / (w_1 ... w_31), G_63 = w_32 ... w_63); beyond that R~ or K~
+        // could leave the float range. Flag it rather than return infinities silently.
+        if (!(G[j] <= 0x1p60f)) atomicOr(err, kErrRange);
+      }
     } else {
+      const float f = qtr == 3 ? q2 : 1.f;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) G[(32 + t) * kGP + j] = p[t];
-      g63[j] = p[31];
-      if (!(p[31] >= 0x1p-60f)) atomicOr(err, kErrRange);
+      for (int t = 0; t < 16; ++t) G[(16 * qtr + t) * kGP + j] = __fmul_rn(f, p[t]);
+      if (qtr == 3) {
+        const float g = __fmul_rn(q2, p[15]);
+        g63[j] = g;
+        if (!(g >= 0x1p-60f)) atomicOr(err, kErrRange);
+      }
     }
   }
   __syncthreads();
@@ -267,8 +297,10 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
     const float4 gg = *reinterpret_cast<const float4*>(G + row * kGP + col);
     const Split4 rs4 = split4(make_float4(__fmul_rn(rr[it].x, gg.x), __fmul_rn(rr[it].y, gg.y),
                                           __fmul_rn(rr[it].z, gg.z), __fmul_rn(rr[it].w, gg.w)));
-    const Split4 ks4 = split4(make_float4(__fdiv_rn(kk[it].x, gg.x), __fdiv_rn(kk[it].y, gg.y),
-                                          __fdiv_rn(kk[it].z, gg.z), __fdiv_rn(kk[it].w, gg.w)));
+    const Split4 ks4 = split4(make_float4(__fmul_rn(kk[it].x, __frcp_rn(gg.x)),
+                                          __fmul_rn(kk[it].y, __frcp_rn(gg.y)),
+                                          __fmul_rn(kk[it].z, __frcp_rn(gg.z)),
+                                          __fmul_rn(kk[it].w, __frcp_rn(gg.w))));
     st_row4(sR, row, col, rs4);
     st_row4(sK, row, col, ks4);
     st_col4(sKt, col, row, ks4);
@@ -283,8 +315,6 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
   fence_proxy_async_smem();
   __syncthreads();
 
-  const uint32_t sb = smem_u32(smem);
-  const uint32_t aR = sb + kOffR, aK = sb + kOffK, aKt = sb + kOffKt, aV = sb + kOffV;
   if (tid == 0) {
     tc_fence_after();
     mma_split(tm + 0, aR, aK, false);     // D_A = R~ K~^T
@@ -296,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
   // + 15 of an M = 64 result in its lanes 0-15) and the column half w / 4.
   const int sub = warp & 3, ch = warp >> 2;
   const int ri = 16 * sub + (lane & 15);
-  const bool act = lane < 16;
+  const int c8 = (lane >> 4) * 8;  // this lane's 8 of each 16 columns (half_row)
   const uint32_t trow = tm + (uint32_t(32 * sub) << 16);
   const float* sprev = c == 0 ? (s0 ? s0 + int64_t(bh) * kHN * kHN : nullptr)
                               : ring + (int64_t(bh) * 2 + ((c - 1) & 1)) * kHN * kHN;
@@ -307,14 +337,15 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
   // guarantees that CTA has started), or the caller's initial state.
   if (c > 0 && tid == 0) wait_flag(flags + bh, unsigned(c), wait_ns, err);
   __syncthreads();
-  float4 sp[8];  // this lane's row of S_{c-1}, its column half
+  float4 sp[4];  // this lane's 8 columns of each 16 (half_row) of its row of S_{c-1}
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    sp[e] = (act && sprev)
-                ? __ldcg(reinterpret_cast<const float4*>(sprev + ri * kHN + 32 * ch + 4 * e))
-                : zero4;
-  mbar_wait(&bar, phase, err);
+  for (int e = 0; e < 4; ++e)
+    sp[e] = sprev ? __ldcg(reinterpret_cast<const float4*>(
+                        sprev + ri * kHN + 32 * ch + 16 * (e >> 1) + c8 + 4 * (e & 1)))
+                  : zero4;
+  if (warp == 0) mbar_wait(&bar, phase, err);  // the others sleep at the barrier
   phase ^= 1u;
+  __syncthreads();
   tc_fence_after();
 
   // S_c = S_{c-1} o gamma_L + D_U o G_63 (gamma_L = gamma_m G_63), stored and published;
@@ -322,26 +353,43 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
     const int q = 2 * ch + qq;
-    float du[16];
-    tmem_ld16_pair(trow + 128 + 16 * q, du);
-    if (act) {
+    float v16[16], du[8];
+    tmem_ld16_pair(trow + 128 + 16 * q, v16);
+    half_row(v16, du, lane);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 16 * q + 4 * e;
-        const float4 x = sp[4 * qq + e];
-        const float4 g = *reinterpret_cast<const float4*>(g63 + j);
-        const float4 m = *reinterpret_cast<const float4*>(gref + j);
-        if (snext) {
-          const float4 sn = make_float4(
-              fmaf(x.x, __fmul_rn(m.x, g.x), __fmul_rn(du[4 * e + 0], g.x)),
-              fmaf(x.y, __fmul_rn(m.y, g.y), __fmul_rn(du[4 * e + 1], g.y)),
-              fmaf(x.z, __fmul_rn(m.z, g.z), __fmul_rn(du[4 * e + 2], g.z)),
-              fmaf(x.w, __fmul_rn(m.w, g.w), __fmul_rn(du[4 * e + 3], g.w)));
-          __stcg(reinterpret_cast<float4*>(snext + ri * kHN + j), sn);
-        }
-        st_row4(sK, ri, j, split4(make_float4(__fmul_rn(x.x, m.x), __fmul_rn(x.y, m.y),
-                                              __fmul_rn(x.z, m.z), __fmul_rn(x.w, m.w))));
+    for (int e = 0; e < 2; ++e) {
+      const int j = 16 * q + c8 + 4 * e;
+      const float4 x = sp[2 * qq + e];
+      const float4 g = *reinterpret_cast<const float4*>(g63 + j);
+      const float4 m = *reinterpret_cast<const float4*>(gref + j);
+      if (snext) {
+        const float4 sn = make_float4(
+            fmaf(x.x, __fmul_rn(m.x, g.x), __fmul_rn(du[4 * e + 0], g.x)),
+            fmaf(x.y, __fmul_rn(m.y, g.y), __fmul_rn(du[4 * e + 1], g.y)),
+            fmaf(x.z, __fmul_rn(m.z, g.z), __fmul_rn(du[4 * e + 2], g.z)),
+            fmaf(x.w, __fmul_rn(m.w, g.w), __fmul_rn(du[4 * e + 3], g.w)));
+        __stcg(reinterpret_cast<float4*>(snext + ri * kHN + j), sn);
       }
+      st_row4(sK, ri, j, split4(make_float4(__fmul_rn(x.x, m.x), __fmul_rn(x.y, m.y),
+                                            __fmul_rn(x.z, m.z), __fmul_rn(x.w, m.w))));
+    }
+  }
+  // A = tril(D_A), split into the K~^T tiles (read no more).
+  const int t_row = ri;
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const int q = 2 * ch + qq;
+    float v16[16], a[8];
+    tmem_ld16_pair(trow + 0 + 16 * q, v16);
+    half_row(v16, a, lane);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int s = 16 * q + c8 + 4 * e;
+      st_row4(sKt, t_row, s,
+              split4(make_float4(s + 0 <= t_row ? a[4 * e + 0] : 0.f,
+                                 s + 1 <= t_row ? a[4 * e + 1] : 0.f,
+                                 s + 2 <= t_row ? a[4 * e + 2] : 0.f,
+                                 s + 3 <= t_row ? a[4 * e + 3] : 0.f)));
     }
   }
   fence_proxy_async_smem();
@@ -352,41 +400,12 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
     st_release(flags + bh, unsigned(c + 1));
     tc_fence_after();
     mma_split(tm + 128, aR, aK, false);   // D_Y = R~ (S_0 o gamma_m)^T
+    mma_split(tm + 128, aKt, aV, true);   //     + A V
     mma_commit(&bar);
   }
-  mbar_wait(&bar, phase, err);
+  if (warp == 0) mbar_wait(&bar, phase, err);  // the others sleep at the barrier
   phase ^= 1u;
-  tc_fence_after();
-
-  // A = tril(D_A), split into the R~ tiles (read no more).
-  const int t_row = ri;
-#pragma unroll
-  for (int qq = 0; qq < 2; ++qq) {
-    const int q = 2 * ch + qq;
-    float a[16];
-    tmem_ld16_pair(trow + 0 + 16 * q, a);
-    if (act) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int s = 16 * q + 4 * e;
-        st_row4(sR, t_row, s,
-                split4(make_float4(s + 0 <= t_row ? a[4 * e + 0] : 0.f,
-                                   s + 1 <= t_row ? a[4 * e + 1] : 0.f,
-                                   s + 2 <= t_row ? a[4 * e + 2] : 0.f,
-                                   s + 3 <= t_row ? a[4 * e + 3] : 0.f)));
-      }
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
   __syncthreads();
-  if (tid == 0) {
-    tc_fence_after();
-    mma_split(tm + 128, aR, aV, true);    // D_Y += A V
-    mma_commit(&bar);
-  }
-  mbar_wait(&bar, phase, err);
-  phase ^= 1u;
   tc_fence_after();
 
   // y rows of this chunk.
@@ -394,12 +413,13 @@ __global__ void __launch_bounds__(kThreads, 2) wkv_mstate_kernel(
 #pragma unroll
   for (int qq = 0; qq < 2; ++qq) {
     const int q = 2 * ch + qq;
-    float o[16];
-    tmem_ld16_pair(trow + 128 + 16 * q, o);
-    if (act && t_row < nvalid) {
+    float v16[16], o[8];
+    tmem_ld16_pair(trow + 128 + 16 * q, v16);
+    half_row(v16, o, lane);
+    if (t_row < nvalid) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        __stcs(reinterpret_cast<float4*>(yrow + 16 * q + 4 * e),
+      for (int e = 0; e < 2; ++e)
+        __stcs(reinterpret_cast<float4*>(yrow + 16 * q + c8 + 4 * e),
                make_float4(o[4 * e + 0], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]));
     }
   }
