@@ -635,7 +635,7 @@ def run_workload(args):
         line("long_ctx", f"forward_state fp32 1x{x.T}x4096 (chunked kernel, final state)", ms, n,
              16 * n + 12 * x.B * x.C)
     elif args.workload == "decode":
-        dd = wkv_inputs.decode_batch(seed=0)
+        dd = wkv_inputs.decode_batch(seed=0, N=args.decode_seqs)
         n = dd.N * dd.L * dd.C
         w, u = d(dd.w), d(dd.u)
         a, b, p = d(dd.a), d(dd.b), d(dd.p)
@@ -643,11 +643,11 @@ def run_workload(args):
         y = torch.empty_like(k)
         ms = _time_loop(lambda: W.wkv_decode_step(w, u, k, v, r, a, b, p, y=y), args.steps,
                         args.warmup, stream)
-        line("decode", "decode step fp32 256 seq x 32 layers x 4096 (state in place)", ms, n,
+        line("decode", f"decode step fp32 {dd.N} seq x 32 layers x 4096 (state in place)", ms, n,
              40 * n, {"tokens_per_s": dd.N / (ms / 1e3)})
         # S tokens per call with the state kept on chip (wkv_decode_steps): per token
         # 16 bytes per state (k, v, r in, y out) plus the state once per call (24 / S).
-        S = 64
+        S = args.seq or 64
         ks = torch.empty((S,) + tuple(k.shape), device=dev)
         vs, rs = torch.empty_like(ks), torch.empty_like(ks)
         for s_ in range(S):
@@ -659,7 +659,7 @@ def run_workload(args):
         steps = max(3, args.steps // S)
         ms = _time_loop(lambda: W.wkv_decode_steps(w, u, ks, vs, rs, a, b, p, y=ys), steps,
                         3, stream)
-        line("decode", f"decode_steps fp32 256 seq x 32 layers x 4096, {S} tokens per call "
+        line("decode", f"decode_steps fp32 {dd.N} seq x 32 layers x 4096, {S} tokens per call "
              "(state on chip between tokens); ms and rates per token", ms / S, n,
              int(16 * n + 24 * n / S), {"tokens_per_s": dd.N * S / (ms / 1e3),
                                         "ms_per_call": ms, "tokens_per_call": S})
@@ -675,13 +675,15 @@ def run_workload(args):
                                                state_out=s1), args.steps, args.warmup, stream)
         # FP32 work per token and head: sa (N^2 FMA), update (N^2 FMUL + 2 N^2 FMA), y (N^2 FMA)
         flops = 9 * x.N * x.N * x.B * x.T * x.H
-        # FP32 peak from unit counts: 148 SMs x 128 FMA lanes x 2 x the max SM clock
+        # FP32 peak from unit counts: 148 SMs x 128 FMA lanes x 2 x the max SM clock (74.4
+        # TFLOP/s; a development probe of packed FFMA2 chains measured 73.7 at 1965 MHz)
         alu_peak = 148 * 128 * 2 * 1.965e9
         line("rwkv7", f"RWKV-7 recurrence fp32 8x{x.T}x64 heads x 64 (state in and out)", ms, n,
              28 * n + 8 * x.B * x.H * x.N * x.N,
              {"flops": flops, "achieved_TFLOPs": flops / (ms / 1e3) / 1e12,
-              "alu_peak_TFLOPs": alu_peak / 1e12,
-              "alu_frac": flops / (ms / 1e3) / alu_peak})
+              "alu_peak_TFLOPs": alu_peak / 1e12, "alu_peak_measured_TFLOPs": 73.7,
+              "alu_frac": flops / (ms / 1e3) / alu_peak,
+              "alu_frac_of_measured": flops / (ms / 1e3) / 73.7e12})
     elif args.workload == "mstate":
         # Matrix-valued state without the delta term: the chunked tensor-core kernel and the
         # token-by-token recurrence kernel on the same inputs (a = b = 0).
@@ -728,10 +730,14 @@ def main():
                     choices=["bf16_7b", "train_169m", "long_ctx", "decode", "rwkv7", "mstate"],
                     help="bf16_7b (default) prints the benchmark line; the others print "
                          "measurements of the other workloads, one GPU")
+    ap.add_argument("--decode-seqs", type=int, default=256,
+                    help="sequences of the decode workload (default 256, the measured one; "
+                         "fewer for profiler captures)")
     ap.add_argument("--seq", type=int, default=None,
                     help="tokens per sequence (default: the workload's own, 4096 for the "
                          "benchmark; shorter sequences keep the occupancy of the full case "
-                         "for profiler captures)")
+                         "for profiler captures); for decode, tokens per wkv_decode_steps "
+                         "call (default 64)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
