@@ -38,6 +38,14 @@ def W():
     f = W.lib.wkv_forward_state_static
     f.argtypes = [ctypes.c_int64] * 3 + [ctypes.c_void_p] * 13
     f.restype = ctypes.c_int
+    # The first call on a device looks up the array's address (and may load the library's
+    # device code): make it here, so that every test's free-memory check sees a later call.
+    x = wkv_inputs.make_inputs(1, 600, 32, seed=7)
+    w, u, k, v, r = (dev(a) for a in (x.w, x.u, x.k, x.v, x.r))
+    y = torch.empty_like(k)
+    out = [torch.empty((x.B, x.C), device="cuda") for _ in range(3)]
+    assert static_call(W, x.B, x.T, x.C, w, u, k, v, r, y, None, out) == 0
+    assert W.wkv_stream_status() == 0
     return W
 
 
