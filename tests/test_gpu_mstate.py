@@ -145,3 +145,25 @@ def test_mstate_no_tokens_and_arguments(W):
     W.wkv_mstate_forward(z, z, z, z, state=s0, state_out=s1)
     assert W.wkv_stream_status() == 0
     assert torch.equal(s0, s1)
+
+
+def _sampled_heads(x, y, S, picks):
+    """y (B, T, H, N) and S (B, H, N, N) of the listed (b, h) heads against the oracle run
+    on those heads alone (heads are independent)."""
+    for b, h in picks:
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        ref, Sref = oracle.wkv7_recurrent(*(getattr(x, n)[sl] for n in "rwkvab"),
+                                          x.S0[b:b + 1, h:h + 1], want_state=True)
+        close(y[sl].cpu().numpy(), ref, f"y of head ({b}, {h})")
+        close(S[b:b + 1, h:h + 1].cpu().numpy(), Sref, f"state of head ({b}, {h})")
+
+
+def test_mstate_benchmark_shape_sampled(W):
+    # The benchmark's launch: 8 x 4096 tokens x 64 heads (32768 chunks on the persistent
+    # CTAs); 16 seeded heads in full against the oracle.
+    x = inputs(8, 4096, 64, seed=0)
+    y, S = W.wkv_mstate_forward(*(dev(getattr(x, n)) for n in "rwkv"), state=dev(x.S0))
+    assert W.wkv_stream_status() == 0
+    g = np.random.Generator(np.random.PCG64(5))
+    picks = [(int(f) // 64, int(f) % 64) for f in g.choice(8 * 64, 16, replace=False)]
+    _sampled_heads(x, y, S, picks)

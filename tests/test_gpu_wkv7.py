@@ -115,3 +115,19 @@ def test_wkv7_larger_shape_sampled(W):
     y, ST, ref, Sref = run(W, x)
     close(y, ref, "y")
     close(ST, Sref, "state")
+
+
+def test_wkv7_benchmark_shape_sampled(W):
+    # The benchmark's launch: 8 x 4096 tokens x 64 heads; 16 seeded heads in full against
+    # the oracle (heads are independent).
+    x = wkv_inputs.rwkv7_inputs(8, 4096, 64, seed=0)
+    y, S = W.wkv7_forward(*(dev(getattr(x, n)) for n in "rwkvab"), state=dev(x.S0))
+    assert W.wkv_stream_status() == 0
+    g = np.random.Generator(np.random.PCG64(5))
+    for f in g.choice(8 * 64, 16, replace=False):
+        b, h = int(f) // 64, int(f) % 64
+        sl = (slice(b, b + 1), slice(None), slice(h, h + 1))
+        ref, Sref = oracle.wkv7_recurrent(*(getattr(x, n)[sl] for n in "rwkvab"),
+                                          x.S0[b:b + 1, h:h + 1], want_state=True)
+        close(y[sl].cpu().numpy(), ref, f"y of head ({b}, {h})")
+        close(S[b:b + 1, h:h + 1].cpu().numpy(), Sref, f"state of head ({b}, {h})")
