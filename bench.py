@@ -162,6 +162,33 @@ class OraclePool:
         shutil.rmtree(self.dir, ignore_errors=True)
 
 
+class InProcessOracle:
+    """The same interface on one core in this process (when the pool cannot run)."""
+
+    def __init__(self, x, note):
+        self.x, self.cores, self.note = x, 1, note
+
+    def run(self, b, c0, c1):
+        import numpy as np
+
+        import oracle
+        x = self.x
+        k, v, r = (np.ascontiguousarray(a[b:b + 1, :, c0:c1]) for a in (x.k, x.v, x.r))
+        oracle.wkv_recurrent(x.w[c0:c1], x.u[c0:c1], k, v, r)
+        return k.size
+
+    def close(self):
+        pass
+
+
+def oracle_runner(x):
+    """OraclePool on all cores, else InProcessOracle with the reason."""
+    try:
+        return OraclePool(x)
+    except Exception as e:  # noqa: BLE001 - report, do not lose the line
+        return InProcessOracle(x, f"process pool unavailable ({type(e).__name__}: {e})")
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -261,14 +288,9 @@ def cpu_oracle_rate(x, budget_s=20.0):
     until the wall-clock budget is spent (at least one row). Returns (elements per second,
     rows done, cores, note). If the process pool cannot be used (e.g. no room for its
     input files), one row in this process on one core instead, with the reason in note."""
-    try:
-        pool = OraclePool(x)
-    except Exception as e:  # noqa: BLE001 - report, do not lose the benchmark line
-        import oracle
-        t0 = time.perf_counter()
-        oracle.wkv_recurrent(x.w, x.u, x.k[:1], x.v[:1], x.r[:1])
-        dt = time.perf_counter() - t0
-        return x.T * x.C / dt, 1, 1, f"process pool unavailable ({type(e).__name__}: {e})"
+    pool = oracle_runner(x)
+    if not isinstance(pool, OraclePool):
+        budget_s = 0.0  # one row on one core
     try:
         rows = elems = 0
         t0 = time.perf_counter()
@@ -280,7 +302,7 @@ def cpu_oracle_rate(x, budget_s=20.0):
         dt = time.perf_counter() - t0
     finally:
         pool.close()
-    return elems / dt, rows, pool.cores, None
+    return elems / dt, rows, pool.cores, getattr(pool, "note", None)
 
 
 def run_reference(args, rank, world):
@@ -291,7 +313,7 @@ def run_reference(args, rank, world):
 
     import wkv_inputs
     x = wkv_inputs.long_bf16(seed=0, B=1)      # one batch row; steps sample channels of it
-    pool = OraclePool(x)
+    pool = oracle_runner(x)
     try:
         # Size each step so that warm-up + timed steps take about a minute in total.
         t0 = time.perf_counter()
@@ -313,9 +335,10 @@ def run_reference(args, rank, world):
     elems = nchan * x.T
     total = sum(times)
     value = elems * len(times) / total / 1e9
+    how = ("process pool over channel blocks" if isinstance(pool, OraclePool)
+           else f"in this process: {pool.note}")
     sample = (f"per step {nchan} channels x {x.T} tokens of batch row 0 of the B=8,T=4096,"
-              f"C=4096 bf16 workload; fp64 recurrence on {pool.cores} host cores (process pool "
-              "over channel blocks)")
+              f"C=4096 bf16 workload; fp64 recurrence on {pool.cores} host cores ({how})")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
