@@ -44,6 +44,15 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
 WKV_API int wkv_testing_backward_timeout(uint64_t wait_ns, cudaStream_t stream);
 
 /*
+ * Chooses the reverse pass of the backward's TMA path for every later call in this process
+ * (wkv_backward, wkv_backward_state, wkv_backward_checkpointed): 0 automatic (one CTA per
+ * channel group when there are at least twice as many groups (batch row x 32 channels) as
+ * SMs, else time-parallel segments), 1 always time-parallel segments, 2 always one CTA per
+ * channel group. Lets tests run both on the same inputs. Other values: WKV_ERR_INVALID_ARG.
+ */
+WKV_API int wkv_testing_set_backward_path(int path);
+
+/*
  * Forces the backward's plain (non-TMA) tile movement; otherwise as wkv_backward.
  */
 WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const float* w,

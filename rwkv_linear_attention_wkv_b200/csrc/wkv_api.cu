@@ -485,6 +485,12 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
   return launch_fwd_stream(a, bf16 != 0, /*force_plain=*/true, stream);
 }
 
+WKV_API int wkv_testing_set_backward_path(int path) {
+  if (path < 0 || path > 2) return WKV_ERR_INVALID_ARG;
+  set_backward_path(path);
+  return WKV_OK;
+}
+
 WKV_API int wkv_testing_backward_plain(int64_t B, int64_t T, int64_t C, const float* w,
                                        const float* u, const float* k, const float* v,
                                        const float* r, const float* dy, float* dk, float* dv,

@@ -44,6 +44,7 @@
 //   3. reduce: dw[c], du[c] = sums of the partials over b and t in a fixed order
 //      (deterministic).
 #include <algorithm>
+#include <atomic>
 
 #include "wkv_internal.h"
 #include "wkv_async.cuh"
@@ -1303,6 +1304,163 @@ __global__ void __launch_bounds__(kSW * 32, 5)
   __syncwarp();
 }
 
+// ---- 2'. reverse pass, one persistent CTA per channel group -----------------------------
+// When there are more channel groups (batch row x 32 channels) than a wave of the
+// time-parallel pass needs to fill the GPU, one CTA per group walks the group's segments
+// from the last to the first: kSW warps recompute and reverse the segment's kSW chunks in
+// parallel, as in wkv_bwd_seg_kernel, but the carry at the segment's end comes from the
+// previous iteration in shared memory. No tickets, no published maps, no waits on other
+// CTAs. The next segment's tiles are brought into L2 while this one is worked on. The
+// per-segment partial sums of dw, du go to the same place as the time-parallel pass's, so
+// the same fixed-order reduction follows.
+template <bool GATE, bool DR, bool FWD>
+__global__ void __launch_bounds__(kSW * 32, 4)
+    wkv_bwd_group_kernel(const __grid_constant__ TensorMaps4 in_maps,
+                         const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
+                         const float* __restrict__ w, const float* __restrict__ u,
+                         const StateIO io, void* ws, unsigned* err, const Ptr4 pre) {
+  constexpr int kTile = kTT * 32;
+  constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
+  extern __shared__ __align__(128) float dyn_tiles[];
+  __shared__ float4 sagg[kSW][32][2];  // the chunks' reverse maps
+  __shared__ float4 sxe[2][32];        // the carry at the segment's end (double-buffered)
+  __shared__ float2 spart[kSW][32];    // the chunks' partial sums (-dw, du)
+  __shared__ uint64_t bars[kSW];
+
+  const int G = (C + 31) >> 5;
+  const int nch = (T + kTT - 1) / kTT;
+  const int nseg = (nch + kSW - 1) / kSW;
+  const BwdLayout lay = bwd_layout(ws, B, T, C);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = int(blockIdx.x) / G, g = int(blockIdx.x) % G;
+  const int c = (g << 5) + lane;
+  const bool valid = c < C;
+  const int64_t sidx = int64_t(b) * C + c;
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, valid ? u[c] : 0.f);
+  const bool fast = __all_sync(0xffffffffu, fabsf(cp.uw2) <= kFastOutBound);
+  const int rb = window_tokens(cp.w2, 128.f);
+  float* tiles = dyn_tiles + warp * kNL * kTile;
+  float* K = tiles + lane;
+  float* V = tiles + kTile + lane;
+  float* R = tiles + 2 * kTile + lane;
+  float* DY = tiles + (kNL - 1) * kTile + lane;
+  uint64_t* bar = &bars[warp];
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  // The carry at the end of the sequence (a later loss's gradient, else zero).
+  if (warp == 0) {
+    float2 e = make_float2(0.f, 0.f);
+    if (io.ga1 != nullptr && valid) {
+      const float4 q = lay.ckend[sidx];
+      e = end_carry(io, sidx, valid, q.z, q.w);
+    }
+    sxe[0][lane] = make_float4(e.x, e.y, 0.f, 0.f);
+  }
+  __syncthreads();
+
+  uint32_t phase = 0;
+  for (int seg = nseg - 1, it = 0; seg >= 0; --seg, ++it) {
+    const int ch = seg * kSW + warp;
+    const bool live = ch < nch;
+    const int t0 = ch * kTT;
+    if (lane == 0 && live) {
+      mbar_arrive_expect_tx(bar, uint32_t(kNL) * kTile * sizeof(float));
+      for (int i = 0; i < kNL; ++i) tma_load_3d(tiles + i * kTile, &in_maps.m[i], bar, g << 5, t0, b);
+    }
+    // the next (earlier) segment's rows of this warp's chunk into L2 meanwhile
+    if (seg > 0) {
+      const int tn = (seg - 1) * kSW * kTT + warp * kTT + (lane & 15);
+      const int64_t off = (int64_t(b) * T + tn) * C + (int64_t(g) << 5);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) prefetch_l2(pre[2 * (lane >> 4) + i] + off);
+    }
+    __syncwarp();
+    const float4 ck = (live && valid) ? lay.ckpt[(int64_t(b) * nch + ch) * C + c]
+                                      : make_float4(0.f, 0.f, kEmptyLogScale, 0.f);
+    const float2 nsc = (live && valid)
+                           ? *reinterpret_cast<const float2*>(
+                                 ch + 1 < nch ? &lay.ckpt[(int64_t(b) * nch + ch + 1) * C + c].z
+                                              : &lay.ckend[sidx].z)
+                           : make_float2(0.f, 0.f);
+    const int nvalid = min(kTT, T - t0);
+
+    // ---- forward recomputation and the chunk's reverse map ----
+    ChunkFactors f;
+    RevAgg A = rev_identity();
+    ChanState s;
+    s.a = ck.x;
+    s.b = ck.y;
+    s.Q = ck.z;
+    s.pl = ck.w;
+    if (live) {
+      mbar_wait_suspend(bar, phase, err);
+      phase ^= 1u;
+      __syncwarp();
+      for (int t = nvalid; t < kTT; ++t) K[t * 32] = -1.0e30f;  // inert positions
+      A = fast ? chunk_forward_rb<GATE, DR, true, FWD>(s, cp, rb, K, V, R, DY, f)
+               : chunk_forward_rb<GATE, DR, false, FWD>(s, cp, rb, K, V, R, DY, f);
+      A.L = float(nvalid);
+    }
+    // the exact ratio between this chunk's recomputed end scale and the next checkpoint's
+    float Ph = s.Q, Pl = s.pl;
+    if (nvalid < kTT) decay_pair(s.Q, s.pl, float(nvalid - kTT), cp.w2, Ph, Pl);
+    const float rme = (live && valid) ? ex2(fminf((Ph - nsc.x) + (Pl - nsc.y), 64.f)) : 1.f;
+    A.E *= rme;
+    put_agg(&sagg[warp][lane][0], A);
+    __syncthreads();
+
+    // ---- the carry at this chunk's end; the carry at the segment's start for the next ----
+    const float4 xe = sxe[it & 1][lane];
+    RevCarry X{xe.x, xe.y, xe.z, xe.w};
+    for (int i = kSW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
+    float dw_init = 0.f;  // the initial state's part of dw (first segment)
+    if (warp == 0) {
+      const RevCarry X0 = rev_apply(A, X);
+      sxe[(it + 1) & 1][lane] = make_float4(X0.b, X0.g, X0.bd, X0.gd);
+      if (seg == 0) {
+        // The carry at the start of the sequence is scaled by the initial state's own
+        // scale (the first checkpoint is that state as given): beta~ = dL/da0.
+        const float a0 = ck.x, b0 = ck.y;
+        if (io.da0 != nullptr && valid) {
+          io.da0[sidx] = X0.b;
+          io.db0[sidx] = -X0.g;
+          io.dp0[sidx] = fmaf(a0, X0.b, -b0 * X0.g);
+        }
+        dw_init = -fmaf(a0, X0.bd, -b0 * X0.gd);
+      }
+    }
+    float2 part = make_float2(0.f, 0.f);
+    if (live) {
+      const RevCarry Xc{X.b * rme, X.g * rme, X.bd * rme, X.gd * rme};
+      part = nvalid == kTT ? chunk_reverse_pairs(f, Xc, K, V, DY)
+                           : chunk_reverse<true>(f, Xc, K, V, DY, nvalid);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        for (int i = 0; i < (DR ? 3 : 2); ++i) tma_store_3d(&out_maps.m[i], tiles + i * kTile, g << 5, t0, b);
+        tma_store_commit();
+      }
+      __syncwarp();
+    }
+    spart[warp][lane] = part;
+    __syncthreads();
+    if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
+      float sw = dw_init, su = 0.f;
+#pragma unroll
+      for (int i = 0; i < kSW; ++i) {
+        sw += spart[i][lane].x;
+        su += spart[i][lane].y;
+      }
+      lay.pdw[(int64_t(b) * nseg + seg) * C + c] = sw;
+      lay.pdu[(int64_t(b) * nseg + seg) * C + c] = su;
+    }
+    if (live && lane == 0) tma_store_wait_read<0>();  // the tiles are reloaded next
+    __syncwarp();
+  }
+}
+
 // ---- 3. reduction over batch rows and segments, fixed order -------------------------------
 // Block (32, kRS): lane x owns a channel; slice y sums the rows y, y + kRS, ... in order,
 // then slice 0 adds the slices' sums in order. Same order on every call: deterministic.
@@ -1372,6 +1530,34 @@ int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, 
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
+// Reverse pass with one CTA per channel group: taken when there are enough groups to fill
+// the GPU (one wave of CTAs at least as wide as the SMs), or when a test forces it.
+std::atomic<int> g_bwd_path{0};  // 0 automatic, 1 time-parallel segments, 2 per group
+
+bool use_group_path(const BwdArgs& a) {
+  const int forced = g_bwd_path.load();
+  if (forced != 0) return forced == 2;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return a.B * ((a.C + 31) / 32) >= 2 * int64_t(sms);
+}
+
+template <bool GATE, bool DR>
+int launch_group(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
+                 cudaStream_t stream) {
+  auto kern = a.have_ckpt ? wkv_bwd_group_kernel<GATE, DR, true>
+                          : wkv_bwd_group_kernel<GATE, DR, false>;
+  const size_t smem = size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+      cudaSuccess)
+    return WKV_ERR_CUDA;
+  const Ptr4 pre{a.k, a.v, a.r ? a.r : a.dy, a.dy};
+  kern<<<unsigned(a.B * ((a.C + 31) / 32)), kSW * 32, smem, stream>>>(
+      in, out, int(a.B), int(a.T), int(a.C), a.w, a.u, state_io(a), a.ws, a.err, pre);
+  return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
 template <bool TMA>
 int launch_all(const BwdArgs& a, cudaStream_t stream) {
   TensorMaps4 ck{}, in{}, out{};
@@ -1401,11 +1587,18 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
           ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
       if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     }
-    if (a.r)
+    if (use_group_path(a) && a.withhold_last_map == 0) {
+      if (a.r)
+        rc = a.dr ? launch_group<true, true>(a, in, out, stream)
+                  : launch_group<true, false>(a, in, out, stream);
+      else
+        rc = launch_group<false, false>(a, in, out, stream);
+    } else if (a.r) {
       rc = a.dr ? launch_seg<true, true>(a, in, out, nitems, stream)
                 : launch_seg<true, false>(a, in, out, nitems, stream);
-    else
+    } else {
       rc = launch_seg<false, false>(a, in, out, nitems, stream);
+    }
   } else {
     wkv_bwd_ckpt_kernel<TMA><<<unsigned(grid), 32, 0, stream>>>(ck, a.k, a.v, int(a.B), int(a.T),
                                                                 int(a.C), a.w, state_io(a), a.ws,
@@ -1466,6 +1659,8 @@ bool backward_time_parallel_ok(const BwdArgs& a) {
   return a.C % 4 == 0 && al16(a.k) && al16(a.v) && al16(a.r) && al16(a.dy) && al16(a.dk) &&
          al16(a.dv) && al16(a.dr);
 }
+
+void set_backward_path(int path) { g_bwd_path.store(path); }
 
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream) {
   const bool tma = !force_plain && backward_time_parallel_ok(a);

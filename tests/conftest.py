@@ -26,3 +26,14 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(params=[1, 2], ids=["segments", "per_group"])
+def bwd_path(request):
+    """Runs a backward test on both reverse passes of the TMA path: the time-parallel
+    segments (1) and one CTA per channel group (2), whatever the automatic choice for the
+    shape would be; back to automatic (0) afterwards."""
+    import rwkv_linear_attention_wkv_b200 as W
+    assert W.lib.wkv_testing_set_backward_path(request.param) == 0
+    yield request.param
+    W.lib.wkv_testing_set_backward_path(0)

@@ -11,7 +11,7 @@ import wkv_inputs
 from wkv_check import assert_fp32_close, assert_grad_close
 
 torch = pytest.importorskip("torch")
-pytestmark = pytest.mark.gpu
+pytestmark = [pytest.mark.gpu, pytest.mark.usefixtures("bwd_path")]
 
 
 @pytest.fixture(scope="module")
