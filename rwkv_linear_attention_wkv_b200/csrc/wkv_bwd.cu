@@ -528,6 +528,109 @@ __global__ void __launch_bounds__(kSW * 32, 6) wkv_bwd_ckpt_seg_kernel(
   if (warp == 0 && first) warp_publish(&lay.fflags[item], 2u);  // the first checkpoint is written
 }
 
+// ---- 1'. checkpoints, one persistent CTA per channel group --------------------------------
+// The counterpart of wkv_bwd_group_kernel for the checkpoint pass: one CTA per channel
+// group walks the group's checkpoint segments (kSW warps x kCK chunks) in order; the warps
+// form their chunks' aggregates from the empty state in parallel, then write the
+// checkpoints from the state entering the segment, which comes from the previous iteration
+// in shared memory (the initial state for the first). No tickets, flags or waits on other
+// CTAs.
+__global__ void __launch_bounds__(kSW * 32, 4) wkv_bwd_ckpt_group_kernel(
+    const __grid_constant__ TensorMaps4 maps, int B, int T, int C, const float* __restrict__ w,
+    const StateIO io, void* ws, unsigned* err, const Ptr4 pre) {
+  constexpr int kTile = kTT * 32;
+  constexpr int kSegC = kSW * kCK;  // chunks per checkpoint segment
+  __shared__ __align__(128) float tiles[kSW][kCK][2][kTile];  // k, v of each warp's chunks
+  __shared__ float4 sagg[kSegC][32];
+  __shared__ float4 sin_[2][32];  // the state entering the segment (double-buffered)
+  __shared__ uint64_t bars[kSW];
+
+  const int G = (C + 31) >> 5;
+  const int nch = (T + kTT - 1) / kTT;
+  const int nseg = (nch + kSegC - 1) / kSegC;
+  const BwdLayout lay = bwd_layout(ws, B, T, C);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = int(blockIdx.x) / G, g = int(blockIdx.x) % G;
+  const int c = (g << 5) + lane;
+  const bool valid = c < C;
+  float4* ck = lay.ckpt + int64_t(b) * nch * C + c;  // checkpoint of chunk i at ck[i * C]
+  const ChanParams cp = chan_params(valid ? w[c] : 1.f, 0.f);
+  const int rb = window_tokens(cp.w2, 128.f);
+  uint64_t* bar = &bars[warp];
+  if (lane == 0) {
+    mbar_init(bar, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    const Agg X = to_agg(initial_state(io, int64_t(b) * C + c, valid));
+    sin_[0][lane] = make_float4(X.a, X.b, X.ph, X.pl);
+  }
+  __syncthreads();
+
+  uint32_t phase = 0;
+  for (int seg = 0; seg < nseg; ++seg) {
+    const int ch0 = seg * kSegC + warp * kCK;  // this warp's first chunk
+    const int nc = max(0, min(kCK, nch - ch0));
+    if (lane == 0 && nc > 0) {
+      fence_proxy_async_smem();  // the previous segment's reads of these tiles come first
+      mbar_arrive_expect_tx(bar, uint32_t(nc) * 2u * kTile * sizeof(float));
+      for (int q = 0; q < nc; ++q) {
+        tma_load_3d(&tiles[warp][q][0][0], &maps.m[0], bar, g << 5, (ch0 + q) * kTT, b);
+        tma_load_3d(&tiles[warp][q][1][0], &maps.m[1], bar, g << 5, (ch0 + q) * kTT, b);
+      }
+    }
+    // the next segment's rows of this warp's chunks into L2 meanwhile
+    if (seg + 1 < nseg) {
+      const int tn = (seg + 1) * kSegC * kTT + warp * kCK * kTT + lane;
+      if (tn < T) {
+        const int64_t off = (int64_t(b) * T + tn) * C + (int64_t(g) << 5);
+        prefetch_l2(pre[0] + off);
+        prefetch_l2(pre[1] + off);
+      }
+    }
+    __syncwarp();
+    if (nc > 0) {
+      mbar_wait_suspend(bar, phase, err);
+      phase ^= 1u;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < kCK; ++q) {
+      const int n = max(0, min(kTT, T - (ch0 + q) * kTT));  // tokens of the chunk
+      Agg A = agg_empty();
+      if (n > 0) {
+        const float* K = &tiles[warp][q][0][lane];
+        const float* V = &tiles[warp][q][1][lane];
+        A = rb == 16 ? chunk_aggregate<16>(K, V, n, cp)
+                     : (rb == 4 ? chunk_aggregate<4>(K, V, n, cp) : chunk_aggregate<1>(K, V, n, cp));
+      }
+      sagg[warp * kCK + q][lane] = make_float4(A.a, A.b, A.ph, A.pl);
+    }
+    __syncthreads();
+
+    // ---- checkpoints; the last warp hands the state after the segment on ----
+    const float4 q = sin_[seg & 1][lane];
+    Agg X{q.x, q.y, q.z, q.w};
+    for (int i = 0; i < warp * kCK; ++i) {  // chunks before this warp's (full)
+      const float4 a = sagg[i][lane];
+      X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(kTT), cp.w2);
+    }
+#pragma unroll
+    for (int q2 = 0; q2 < kCK; ++q2) {
+      const int chq = ch0 + q2;
+      if (chq < nch) {
+        if (valid) ck[int64_t(chq) * C] = make_float4(X.a, X.b, X.ph, X.pl);
+        const float4 a = sagg[warp * kCK + q2][lane];
+        X = combine(X, Agg{a.x, a.y, a.z, a.w}, float(min(kTT, T - chq * kTT)), cp.w2);
+        // after the last chunk: the state after the last token
+        if (chq + 1 == nch && valid) lay.ckend[int64_t(b) * C + c] = make_float4(X.a, X.b, X.ph, X.pl);
+      }
+    }
+    if (warp == kSW - 1) sin_[(seg + 1) & 1][lane] = make_float4(X.a, X.b, X.ph, X.pl);
+    __syncthreads();
+  }
+}
+
 // ---- 2. reverse pass ---------------------------------------------------------------------
 // Shared memory per CTA (floats): kMS stages x 4 tiles (k, v, r, dy; dk, dv, dr written in
 // place of k, v, r) + 6 factor tiles (e1, e2, f_inj, f_cur, wkv, sigma).
@@ -1583,8 +1686,14 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     if (!a.have_ckpt) {
       const int64_t nch = (a.T + kTT - 1) / kTT;
       const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
-      wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
-          ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
+      if (use_group_path(a)) {
+        const Ptr4 pre{a.k, a.v, a.k, a.v};
+        wkv_bwd_ckpt_group_kernel<<<unsigned(grid), kSW * 32, 0, stream>>>(
+            ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, pre);
+      } else {
+        wkv_bwd_ckpt_seg_kernel<<<unsigned(citems), kSW * 32, 0, stream>>>(
+            ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, a.wait_ns);
+      }
       if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     }
     if (use_group_path(a) && a.withhold_last_map == 0) {
