@@ -72,7 +72,9 @@ struct BwdLayout {
   unsigned* rticket;  // segment tickets of the reverse pass (reverse chain)
   unsigned* fflags;   // [nbg * nseg']: 1 once the checkpoint segment's aggregate is published,
                       // 2 once the state entering it (its first checkpoint) is written
-                      // (nseg' <= nseg checkpoint segments of kSW kCK chunks)
+                      // (nseg' <= nseg checkpoint segments of kSW kCK chunks); on the
+                      // per-group path its first G words count the batch rows done per
+                      // channel group instead
   unsigned* rflags;   // [nbg * nseg]: 1 once the segment's reverse map is published, 2 its carry
   float4* fagg;      // [nbg * nseg', 32]: the checkpoint segment's aggregate (a, b, ph, pl)
   float4* rmap;      // [nbg * nseg, 32, 2]: the segment's reverse map (see RevAgg)
@@ -565,6 +567,8 @@ __global__ void __launch_bounds__(kSW * 32, 4) wkv_bwd_ckpt_group_kernel(
     const Agg X = to_agg(initial_state(io, int64_t(b) * C + c, valid));
     sin_[0][lane] = make_float4(X.a, X.b, X.ph, X.pl);
   }
+  // the reverse pass that follows counts the batch rows done per channel group from zero
+  if (b == 0 && threadIdx.x == 0) lay.fflags[g] = 0u;
   __syncthreads();
 
   uint32_t phase = 0;
@@ -1413,15 +1417,17 @@ __global__ void __launch_bounds__(kSW * 32, 5)
 // from the last to the first: kSW warps recompute and reverse the segment's kSW chunks in
 // parallel, as in wkv_bwd_seg_kernel, but the carry at the segment's end comes from the
 // previous iteration in shared memory. No tickets, no published maps, no waits on other
-// CTAs. The next segment's tiles are brought into L2 while this one is worked on. The
-// per-segment partial sums of dw, du go to the same place as the time-parallel pass's, so
-// the same fixed-order reduction follows.
+// CTAs. The next segment's tiles are brought into L2 while this one is worked on. The CTA
+// adds its segments' partial sums of dw, du in a fixed order (last segment first) into one
+// row per batch row; the last CTA of a channel group to finish (a counter per group, zero
+// on entry) adds the group's rows in batch order and writes dw, du: no reduction kernel.
 template <bool GATE, bool DR, bool FWD>
 __global__ void __launch_bounds__(kSW * 32, 4)
     wkv_bwd_group_kernel(const __grid_constant__ TensorMaps4 in_maps,
                          const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
                          const float* __restrict__ w, const float* __restrict__ u,
-                         const StateIO io, void* ws, unsigned* err, const Ptr4 pre) {
+                         const StateIO io, void* ws, unsigned* err, const Ptr4 pre,
+                         float* __restrict__ dw, float* __restrict__ du) {
   constexpr int kTile = kTT * 32;
   constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
   extern __shared__ __align__(128) float dyn_tiles[];
@@ -1464,6 +1470,7 @@ __global__ void __launch_bounds__(kSW * 32, 4)
   __syncthreads();
 
   uint32_t phase = 0;
+  float tw = 0.f, tu = 0.f;  // warp 0: this batch row's sums of -dw, du so far
   for (int seg = nseg - 1, it = 0; seg >= 0; --seg, ++it) {
     const int ch = seg * kSW + warp;
     const bool live = ch < nch;
@@ -1549,18 +1556,43 @@ __global__ void __launch_bounds__(kSW * 32, 4)
     }
     spart[warp][lane] = part;
     __syncthreads();
-    if (warp == 0 && valid) {  // the segment's partial sums, chunks in a fixed order
+    if (warp == 0) {  // the segment's partial sums, chunks in a fixed order
       float sw = dw_init, su = 0.f;
 #pragma unroll
       for (int i = 0; i < kSW; ++i) {
         sw += spart[i][lane].x;
         su += spart[i][lane].y;
       }
-      lay.pdw[(int64_t(b) * nseg + seg) * C + c] = sw;
-      lay.pdu[(int64_t(b) * nseg + seg) * C + c] = su;
+      tw += sw;
+      tu += su;
     }
     if (live && lane == 0) tma_store_wait_read<0>();  // the tiles are reloaded next
     __syncwarp();
+  }
+  // ---- this batch row's sums; the group's last CTA adds the rows and writes dw, du ----
+  if (warp == 0) {
+    if (valid) {
+      __stcg(&lay.pdw[int64_t(b) * nseg * C + c], tw);
+      __stcg(&lay.pdu[int64_t(b) * nseg * C + c], tu);
+    }
+    __threadfence();  // the row is visible before the count says so
+    __syncwarp();
+    unsigned done = 0;
+    if (lane == 0) done = atomicAdd(&lay.fflags[g], 1u);
+    done = __shfl_sync(0xffffffffu, done, 0);
+    if (done == unsigned(B) - 1u) {
+      __threadfence();  // every other row is visible after the count that said so
+      float sw = 0.f, su = 0.f;
+      if (valid)
+        for (int bb = 0; bb < B; ++bb) {
+          sw += __ldcg(&lay.pdw[int64_t(bb) * nseg * C + c]);
+          su += __ldcg(&lay.pdu[int64_t(bb) * nseg * C + c]);
+        }
+      if (valid) {
+        dw[c] = sw;
+        du[c] = su;
+      }
+    }
   }
 }
 
@@ -1657,7 +1689,8 @@ int launch_group(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out
     return WKV_ERR_CUDA;
   const Ptr4 pre{a.k, a.v, a.r ? a.r : a.dy, a.dy};
   kern<<<unsigned(a.B * ((a.C + 31) / 32)), kSW * 32, smem, stream>>>(
-      in, out, int(a.B), int(a.T), int(a.C), a.w, a.u, state_io(a), a.ws, a.err, pre);
+      in, out, int(a.B), int(a.T), int(a.C), a.w, a.u, state_io(a), a.ws, a.err, pre, a.dw,
+      a.du);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
 }
 
@@ -1677,16 +1710,26 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     ck.m[1] = in.m[1];
   }
   int rc;
+  const bool group = TMA && use_group_path(a) && a.withhold_last_map == 0;
   if (TMA) {
     // Time-parallel checkpoints and reverse: the chain flags and the tickets start at zero.
+    // Per-group path: only the counters of batch rows done per channel group, which the
+    // per-group checkpoint pass clears when it runs.
     const int64_t nitems = grid * bwd_nseg(a.T);
     if (nitems >= (int64_t(1) << 31)) return WKV_ERR_UNSUPPORTED;
-    if (cudaMemsetAsync(a.ws, 0, bwd_flag_bytes(a.B, a.T, a.C), stream) != cudaSuccess)
-      return WKV_ERR_CUDA;
+    if (!group) {
+      if (cudaMemsetAsync(a.ws, 0, bwd_flag_bytes(a.B, a.T, a.C), stream) != cudaSuccess)
+        return WKV_ERR_CUDA;
+    } else if (a.have_ckpt) {
+      const BwdLayout lay = bwd_layout(a.ws, a.B, a.T, a.C);
+      if (cudaMemsetAsync(lay.fflags, 0, size_t((a.C + 31) / 32) * sizeof(unsigned), stream) !=
+          cudaSuccess)
+        return WKV_ERR_CUDA;
+    }
     if (!a.have_ckpt) {
       const int64_t nch = (a.T + kTT - 1) / kTT;
       const int64_t citems = grid * ((nch + kSW * kCK - 1) / (kSW * kCK));
-      if (use_group_path(a)) {
+      if (group) {
         const Ptr4 pre{a.k, a.v, a.k, a.v};
         wkv_bwd_ckpt_group_kernel<<<unsigned(grid), kSW * 32, 0, stream>>>(
             ck, int(a.B), int(a.T), int(a.C), a.w, state_io(a), a.ws, a.err, pre);
@@ -1696,7 +1739,7 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
       }
       if (cudaPeekAtLastError() != cudaSuccess) return WKV_ERR_CUDA;
     }
-    if (use_group_path(a) && a.withhold_last_map == 0) {
+    if (group) {
       if (a.r)
         rc = a.dr ? launch_group<true, true>(a, in, out, stream)
                   : launch_group<true, false>(a, in, out, stream);
@@ -1719,7 +1762,7 @@ int launch_all(const BwdArgs& a, cudaStream_t stream) {
     else
       rc = launch_main<TMA, false, false>(a, in, out, stream);
   }
-  if (rc) return rc;
+  if (rc || group) return rc;  // (the per-group reverse pass writes dw, du itself)
   wkv_bwd_reduce_kernel<<<unsigned((a.C + 31) / 32), dim3(32, kRS), 0, stream>>>(
       int(a.B), int(a.C), a.ws, int(a.T), a.dw, a.du);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
