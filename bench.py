@@ -656,6 +656,15 @@ def run_workload(args):
         line("train_169m", "training step: wkv_forward + wkv_backward", ms_p, n, 16 * n + 28 * n)
         line("train_169m", "training step: wkv_forward_checkpointed + wkv_backward_checkpointed",
              ms_c, n, 17 * n + 29 * n)
+        # The same step captured once in a CUDA graph and replayed: no host work and no
+        # launch gaps between the kernels.
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step_ckpt()
+        ms_g = _time_loop(graph.replay, args.steps, args.warmup, stream)
+        line("train_169m", "training step: the checkpointed pair replayed from a CUDA graph",
+             ms_g, n, 17 * n + 29 * n)
+        del graph
     elif args.workload == "long_ctx":
         x = wkv_inputs.long_context(seed=0, T=args.seq or 32768)
         w, u, k, v, r = (d(a) for a in (x.w, x.u, x.k, x.v, x.r))
