@@ -26,23 +26,29 @@
 // and the scale is the forward's exact windowed one, so nothing drifts.
 //
 // Two passes plus a reduction:
-//   1. checkpoints: the state entering every chunk of kTT tokens. Time-parallel on TMA
-//      shapes (wkv_bwd_ckpt_seg_kernel: chunk aggregates folded across segments, in the
-//      state-independent token weights of wkv_indep.cuh); serially otherwise
-//      (wkv_bwd_ckpt_kernel: one warp per 32 channels walks the sequence in the streaming
-//      forward's arithmetic). In the checkpointed training pair the forward has written
-//      them already (the streaming kernel's checkpointing mode) and this pass is skipped;
-//   2. reverse, time-parallel (TMA shapes): one warp per chunk recomputes the chunk's
-//      forward from its checkpoint (in the arithmetic that made the checkpoint: the
-//      template flag FWD), the carries of the reverse sums are chained across segments of
-//      kSW chunks, and each warp then runs the reverse over its chunk (see section 2'
-//      below). Shapes TMA cannot address take the serial form: one warp per 32 channels
-//      walks the chunks from last to first, recomputing each chunk's factors into shared
-//      memory before its reverse;
+//   1. checkpoints: the state entering every chunk of kTT tokens. On TMA shapes either
+//      time-parallel (wkv_bwd_ckpt_seg_kernel: chunk aggregates folded across segments, in
+//      the state-independent token weights of wkv_indep.cuh) or, when the channel groups
+//      (batch row x 32 channels) number at least twice the SMs, one persistent CTA per
+//      group walking its segments in order (wkv_bwd_ckpt_group_kernel); serially on other
+//      shapes (wkv_bwd_ckpt_kernel: one warp per 32 channels walks the sequence in the
+//      streaming forward's arithmetic). In the checkpointed training pair the forward has
+//      written them already (the streaming kernel's checkpointing mode) and this pass is
+//      skipped;
+//   2. reverse (TMA shapes): one warp per chunk recomputes the chunk's forward from its
+//      checkpoint (in the arithmetic that made the checkpoint: the template flag FWD) and
+//      then runs the reverse over its chunk. The carry at each segment's end (kSW chunks)
+//      is either chained across CTAs through published maps (wkv_bwd_seg_kernel,
+//      time-parallel) or, with as many groups as above, kept on chip by one persistent CTA
+//      per group walking its segments from the last (wkv_bwd_group_kernel). Shapes TMA
+//      cannot address take the serial form: one warp per 32 channels walks the chunks from
+//      last to first, recomputing each chunk's factors into shared memory before its
+//      reverse;
 //   both write dk, dv (dr) in place of k, v (r) in shared memory for the stores, and
-//   per-(b, segment or chunk, c) partial sums of dw, du to the workspace;
+//   partial sums of dw, du to the workspace;
 //   3. reduce: dw[c], du[c] = sums of the partials over b and t in a fixed order
-//      (deterministic).
+//      (deterministic): a kernel of its own (wkv_bwd_reduce_kernel), or, on the per-group
+//      path, the last reverse-pass CTA of each channel group.
 #include <algorithm>
 #include <atomic>
 
