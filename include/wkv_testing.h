@@ -1,6 +1,8 @@
 /*
  * wkv_testing.h — test hooks of libwkv.so. Not part of the operator: these entry points
- * exist so that the library's failure handling can be exercised without faulting a GPU.
+ * exist so that the library's failure handling can be exercised without faulting a GPU,
+ * so that tests can force one path or another, and so that the rooflines' compute
+ * denominators can be measured on the GPU at hand.
  */
 #ifndef WKV_TESTING_H_
 #define WKV_TESTING_H_
@@ -70,6 +72,24 @@ WKV_API int wkv_testing_backward_state_plain(
     const float* p0, const float* ga1, const float* gb1, const float* p1, float* dk, float* dv,
     float* dw, float* du, float* dr, float* da0, float* db0, float* dp0, void* workspace,
     size_t workspace_bytes, cudaStream_t stream);
+
+/* Pipes wkv_testing_pipe_rate can measure. */
+#define WKV_PIPE_EX2 0   /* ex2.approx.ftz.f32 instructions per second (MUFU) */
+#define WKV_PIPE_FFMA2 1 /* fp32 flops per second through packed fp32x2 FMA (4 per instruction) */
+
+/*
+ * Measures one pipe's throughput on the current device: a grid of 8 CTAs x 256 threads per
+ * SM, each thread running 8 independent chains of `iters` instructions (1 <= iters <=
+ * 2^30), timed with CUDA events on `stream` (the call synchronises on its end event).
+ * Writes the rate to *per_second (host pointer): the denominators of the exponential
+ * (SFU) roofline term of the forward and of the RWKV-7 recurrence's FP32 roofline, as this
+ * GPU sustains them (nominal figures, unit counts x the maximum clock, assume a clock the
+ * power cap does not always allow). Compute only, apart from a one-float buffer it
+ * allocates and frees on `stream` (nothing is ever stored to it).
+ * Returns WKV_ERR_INVALID_ARG for an unknown pipe, out-of-range iters or a null pointer.
+ */
+WKV_API int wkv_testing_pipe_rate(int pipe, int64_t iters, double* per_second,
+                                  cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -54,6 +54,8 @@ _SIGS = {
     "wkv_testing_backward_timeout": ([ctypes.c_uint64, _P], ctypes.c_int),
     "wkv_testing_forward_plain": ([_I, _I, _I] + [_P] * 6 + [ctypes.c_int, _P], ctypes.c_int),
     "wkv_testing_set_backward_path": ([ctypes.c_int], ctypes.c_int),
+    "wkv_testing_pipe_rate": ([ctypes.c_int, _I, ctypes.POINTER(ctypes.c_double), _P],
+                              ctypes.c_int),
 }
 for _name, (_args, _res) in _SIGS.items():
     try:
