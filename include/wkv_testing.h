@@ -50,7 +50,9 @@ WKV_API int wkv_testing_backward_timeout(uint64_t wait_ns, cudaStream_t stream);
  * (wkv_backward, wkv_backward_state, wkv_backward_checkpointed): 0 automatic (one CTA per
  * channel group when there are at least twice as many groups (batch row x 32 channels) as
  * SMs, else time-parallel segments), 1 always time-parallel segments, 2 always one CTA per
- * channel group. Lets tests run both on the same inputs. Other values: WKV_ERR_INVALID_ARG.
+ * channel group (of five warps while the groups number at most three times the SMs, else
+ * four), 3 always one CTA of four warps per channel group. Lets tests run every form on the
+ * same inputs. Other values: WKV_ERR_INVALID_ARG.
  */
 WKV_API int wkv_testing_set_backward_path(int path);
 

@@ -486,7 +486,7 @@ WKV_API int wkv_testing_forward_plain(int64_t B, int64_t T, int64_t C, const flo
 }
 
 WKV_API int wkv_testing_set_backward_path(int path) {
-  if (path < 0 || path > 2) return WKV_ERR_INVALID_ARG;
+  if (path < 0 || path > 3) return WKV_ERR_INVALID_ARG;
   set_backward_path(path);
   return WKV_OK;
 }

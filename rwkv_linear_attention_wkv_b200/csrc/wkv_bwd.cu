@@ -1420,15 +1420,15 @@ __global__ void __launch_bounds__(kSW * 32, 5)
 // ---- 2'. reverse pass, one persistent CTA per channel group -----------------------------
 // When there are more channel groups (batch row x 32 channels) than a wave of the
 // time-parallel pass needs to fill the GPU, one CTA per group walks the group's segments
-// from the last to the first: kSW warps recompute and reverse the segment's kSW chunks in
+// from the last to the first: NW warps recompute and reverse the segment's NW chunks in
 // parallel, as in wkv_bwd_seg_kernel, but the carry at the segment's end comes from the
 // previous iteration in shared memory. No tickets, no published maps, no waits on other
 // CTAs. The next segment's tiles are brought into L2 while this one is worked on. The CTA
 // adds its segments' partial sums of dw, du in a fixed order (last segment first) into one
 // row per batch row; the last CTA of a channel group to finish (a counter per group, zero
 // on entry) adds the group's rows in batch order and writes dw, du: no reduction kernel.
-template <bool GATE, bool DR, bool FWD>
-__global__ void __launch_bounds__(kSW * 32, 4)
+template <bool GATE, bool DR, bool FWD, int NW>
+__global__ void __launch_bounds__(NW * 32, NW <= 4 ? 4 : 3)
     wkv_bwd_group_kernel(const __grid_constant__ TensorMaps4 in_maps,
                          const __grid_constant__ TensorMaps4 out_maps, int B, int T, int C,
                          const float* __restrict__ w, const float* __restrict__ u,
@@ -1437,14 +1437,14 @@ __global__ void __launch_bounds__(kSW * 32, 4)
   constexpr int kTile = kTT * 32;
   constexpr int kNL = GATE ? 4 : 3;  // tiles per chunk: k, v, (r,) dy
   extern __shared__ __align__(128) float dyn_tiles[];
-  __shared__ float4 sagg[kSW][32][2];  // the chunks' reverse maps
+  __shared__ float4 sagg[NW][32][2];  // the chunks' reverse maps
   __shared__ float4 sxe[2][32];        // the carry at the segment's end (double-buffered)
-  __shared__ float2 spart[kSW][32];    // the chunks' partial sums (-dw, du)
-  __shared__ uint64_t bars[kSW];
+  __shared__ float2 spart[NW][32];    // the chunks' partial sums (-dw, du)
+  __shared__ uint64_t bars[NW];
 
   const int G = (C + 31) >> 5;
   const int nch = (T + kTT - 1) / kTT;
-  const int nseg = (nch + kSW - 1) / kSW;
+  const int nseg = (nch + NW - 1) / NW;  // this kernel's segments of NW chunks
   const BwdLayout lay = bwd_layout(ws, B, T, C);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = int(blockIdx.x) / G, g = int(blockIdx.x) % G;
@@ -1478,7 +1478,7 @@ __global__ void __launch_bounds__(kSW * 32, 4)
   uint32_t phase = 0;
   float tw = 0.f, tu = 0.f;  // warp 0: this batch row's sums of -dw, du so far
   for (int seg = nseg - 1, it = 0; seg >= 0; --seg, ++it) {
-    const int ch = seg * kSW + warp;
+    const int ch = seg * NW + warp;
     const bool live = ch < nch;
     const int t0 = ch * kTT;
     if (lane == 0 && live) {
@@ -1487,7 +1487,7 @@ __global__ void __launch_bounds__(kSW * 32, 4)
     }
     // the next (earlier) segment's rows of this warp's chunk into L2 meanwhile
     if (seg > 0) {
-      const int tn = (seg - 1) * kSW * kTT + warp * kTT + (lane & 15);
+      const int tn = (seg - 1) * NW * kTT + warp * kTT + (lane & 15);
       const int64_t off = (int64_t(b) * T + tn) * C + (int64_t(g) << 5);
 #pragma unroll
       for (int i = 0; i < 2; ++i) prefetch_l2(pre[2 * (lane >> 4) + i] + off);
@@ -1530,7 +1530,7 @@ __global__ void __launch_bounds__(kSW * 32, 4)
     // ---- the carry at this chunk's end; the carry at the segment's start for the next ----
     const float4 xe = sxe[it & 1][lane];
     RevCarry X{xe.x, xe.y, xe.z, xe.w};
-    for (int i = kSW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
+    for (int i = NW - 1; i > warp; --i) X = rev_apply(get_agg(sagg[i][lane][0], sagg[i][lane][1]), X);
     float dw_init = 0.f;  // the initial state's part of dw (first segment)
     if (warp == 0) {
       const RevCarry X0 = rev_apply(A, X);
@@ -1565,7 +1565,7 @@ __global__ void __launch_bounds__(kSW * 32, 4)
     if (warp == 0) {  // the segment's partial sums, chunks in a fixed order
       float sw = dw_init, su = 0.f;
 #pragma unroll
-      for (int i = 0; i < kSW; ++i) {
+      for (int i = 0; i < NW; ++i) {
         sw += spart[i][lane].x;
         su += spart[i][lane].y;
       }
@@ -1578,8 +1578,8 @@ __global__ void __launch_bounds__(kSW * 32, 4)
   // ---- this batch row's sums; the group's last CTA adds the rows and writes dw, du ----
   if (warp == 0) {
     if (valid) {
-      __stcg(&lay.pdw[int64_t(b) * nseg * C + c], tw);
-      __stcg(&lay.pdu[int64_t(b) * nseg * C + c], tu);
+      __stcg(&lay.pdw[int64_t(b) * bwd_nseg(T) * C + c], tw);
+      __stcg(&lay.pdu[int64_t(b) * bwd_nseg(T) * C + c], tu);
     }
     __threadfence();  // the row is visible before the count says so
     __syncwarp();
@@ -1591,8 +1591,8 @@ __global__ void __launch_bounds__(kSW * 32, 4)
       float sw = 0.f, su = 0.f;
       if (valid)
         for (int bb = 0; bb < B; ++bb) {
-          sw += __ldcg(&lay.pdw[int64_t(bb) * nseg * C + c]);
-          su += __ldcg(&lay.pdu[int64_t(bb) * nseg * C + c]);
+          sw += __ldcg(&lay.pdw[int64_t(bb) * bwd_nseg(T) * C + c]);
+          su += __ldcg(&lay.pdu[int64_t(bb) * bwd_nseg(T) * C + c]);
         }
       if (valid) {
         dw[c] = sw;
@@ -1673,31 +1673,49 @@ int launch_seg(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out, 
 
 // Reverse pass with one CTA per channel group: taken when there are enough groups to fill
 // the GPU (one wave of CTAs at least as wide as the SMs), or when a test forces it.
-std::atomic<int> g_bwd_path{0};  // 0 automatic, 1 time-parallel segments, 2 per group
+// 0 automatic, 1 time-parallel segments, 2 per group (warps per CTA automatic), 3 per group
+// with 4 warps per CTA.
+std::atomic<int> g_bwd_path{0};
 
-bool use_group_path(const BwdArgs& a) {
-  const int forced = g_bwd_path.load();
-  if (forced != 0) return forced == 2;
+int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return a.B * ((a.C + 31) / 32) >= 2 * int64_t(sms);
+  return sms;
 }
 
-template <bool GATE, bool DR>
-int launch_group(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
-                 cudaStream_t stream) {
-  auto kern = a.have_ckpt ? wkv_bwd_group_kernel<GATE, DR, true>
-                          : wkv_bwd_group_kernel<GATE, DR, false>;
-  const size_t smem = size_t(kSW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
+bool use_group_path(const BwdArgs& a) {
+  const int forced = g_bwd_path.load();
+  if (forced != 0) return forced >= 2;
+  return a.B * ((a.C + 31) / 32) >= 2 * int64_t(sm_count());
+}
+
+template <bool GATE, bool DR, int NW>
+int launch_group_nw(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
+                    cudaStream_t stream) {
+  auto kern = a.have_ckpt ? wkv_bwd_group_kernel<GATE, DR, true, NW>
+                          : wkv_bwd_group_kernel<GATE, DR, false, NW>;
+  const size_t smem = size_t(NW) * (GATE ? 4 : 3) * kTT * 32 * sizeof(float);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
       cudaSuccess)
     return WKV_ERR_CUDA;
   const Ptr4 pre{a.k, a.v, a.r ? a.r : a.dy, a.dy};
-  kern<<<unsigned(a.B * ((a.C + 31) / 32)), kSW * 32, smem, stream>>>(
+  kern<<<unsigned(a.B * ((a.C + 31) / 32)), NW * 32, smem, stream>>>(
       in, out, int(a.B), int(a.T), int(a.C), a.w, a.u, state_io(a), a.ws, a.err, pre, a.dw,
       a.du);
   return cudaPeekAtLastError() == cudaSuccess ? WKV_OK : WKV_ERR_CUDA;
+}
+
+// Five warps (five chunks an iteration, 3 CTAs per SM at 128 registers) while every group's
+// CTA fits in one wave at 3 per SM, else four (4 per SM): measured 76.6 against 79.8 us at
+// 384 groups, 198.7 against 194.8 at 1024.
+template <bool GATE, bool DR>
+int launch_group(const BwdArgs& a, const TensorMaps4& in, const TensorMaps4& out,
+                 cudaStream_t stream) {
+  const bool five = g_bwd_path.load() != 3 &&
+                    a.B * ((a.C + 31) / 32) <= 3 * int64_t(sm_count());
+  return five ? launch_group_nw<GATE, DR, 5>(a, in, out, stream)
+              : launch_group_nw<GATE, DR, 4>(a, in, out, stream);
 }
 
 template <bool TMA>

@@ -132,7 +132,7 @@ bool backward_time_parallel_ok(const BwdArgs& a);
 int launch_fwd_ckpt(const FwdArgs& a, void* ws, cudaStream_t stream);
 int launch_backward(const BwdArgs& a, bool force_plain, cudaStream_t stream);
 // Which reverse pass the TMA path takes: 0 automatic, 1 time-parallel segments, 2 one CTA
-// per channel group (a test hook; process-wide).
+// per channel group, 3 one CTA of four warps per channel group (a test hook; process-wide).
 void set_backward_path(int path);
 // T == 0 with the state's gradients wanted: they pass straight through.
 int launch_backward_no_tokens(const BwdArgs& a, cudaStream_t stream);

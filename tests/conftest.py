@@ -28,7 +28,7 @@ def pytest_collection_modifyitems(config, items):
             item.add_marker(skip)
 
 
-@pytest.fixture(params=[1, 2], ids=["segments", "per_group"])
+@pytest.fixture(params=[1, 2, 3], ids=["segments", "per_group", "per_group_4warps"])
 def bwd_path(request):
     """Runs a backward test on both reverse passes of the TMA path: the time-parallel
     segments (1) and one CTA per channel group (2), whatever the automatic choice for the

@@ -175,3 +175,26 @@ def test_binding_matches_the_declarations(W):
     for name, (args, _) in _SIGS.items():
         assert name in sigs, name
         assert [ctype_kind(a) for a in args] == [kind(t) for t in sigs[name]], name
+
+
+def test_backward_path_hook_values(W):
+    # The test hook that chooses the backward's reverse pass is host-only state: 0..3 are
+    # accepted, anything else is refused, and the automatic choice is restored.
+    f = W.lib.wkv_testing_set_backward_path
+    try:
+        for path in (0, 1, 2, 3):
+            assert f(path) == 0
+        for path in (-1, 4, 100):
+            assert f(path) == 1  # WKV_ERR_INVALID_ARG
+    finally:
+        assert f(0) == 0
+
+
+def test_pipe_probe_argument_checks(W):
+    # Refused before anything touches a device.
+    out = ctypes.c_double(0.0)
+    f = W.lib.wkv_testing_pipe_rate
+    assert f(7, 10, ctypes.byref(out), None) == 1
+    assert f(0, 0, ctypes.byref(out), None) == 1
+    assert f(1, -5, ctypes.byref(out), None) == 1
+    assert f(0, 10, None, None) == 1
