@@ -198,3 +198,21 @@ def test_pipe_probe_argument_checks(W):
     assert f(0, 0, ctypes.byref(out), None) == 1
     assert f(1, -5, ctypes.byref(out), None) == 1
     assert f(0, 10, None, None) == 1
+
+
+def test_binding_refuses_host_tensors_and_wrong_dtypes(W):
+    # The product path has no CPU implementation: the binding refuses host tensors (and
+    # objects that are not tensors) before anything is launched, rather than computing
+    # anywhere else.
+    import torch
+    C = 8
+    w, u = torch.ones(C), torch.zeros(C)
+    k = v = r = torch.zeros(1, 4, C)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        W.wkv_forward(w, u, k, v, r)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        W.wkv_forward_bf16(w, u, k.bfloat16(), v.bfloat16(), r.bfloat16())
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        W.wkv_backward(w, u, k, v, r, k)
+    with pytest.raises(TypeError, match="torch.Tensor"):
+        W.wkv_forward(w, u, k.numpy(), v, r)
