@@ -107,6 +107,14 @@ def _need(t, name, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
+def _dims(t, name, n):
+    """Whether t has n dimensions; t must be a tensor (checked before its shape is read)."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    return t.dim() == n
+
+
 def _call(fn, *args):
     rc = getattr(lib, fn)(*args)
     if rc != 0:
@@ -115,7 +123,7 @@ def _call(fn, *args):
 
 def _fwd_common(w, u, k, v, r, y, dtype):
     torch = _torch()
-    if k.dim() != 3:
+    if not _dims(k, "k", 3):
         raise ValueError("k must be (B, T, C)")
     B, T, C = k.shape
     _need(k, "k", dtype)
@@ -178,7 +186,7 @@ def wkv_forward_state(w, u, k, v, r=None, state=None, y=None, state_out=None,
 def wkv_decode_step(w, u, k, v, r, a, b, p, y=None, stream=None):
     """One token for [N, L, C] states; w, u [L, C]; (a, b, p) updated in place. Returns y."""
     torch = _torch()
-    if k.dim() != 3:
+    if not _dims(k, "k", 3):
         raise ValueError("k must be (N, L, C)")
     N, L, C = k.shape
     f32 = torch.float32
@@ -201,7 +209,7 @@ def wkv_decode_steps(w, u, k, v, r, a, b, p, y=None, stream=None):
     """S chained tokens for [N, L, C] states in one call: k, v, r (S, N, L, C); w, u
     [L, C]; (a, b, p) updated in place. Returns y (S, N, L, C)."""
     torch = _torch()
-    if k.dim() != 4:
+    if not _dims(k, "k", 4):
         raise ValueError("k must be (S, N, L, C)")
     S, N, L, C = k.shape
     f32 = torch.float32
@@ -236,7 +244,7 @@ def wkv_backward(w, u, k, v, r, dy, want_dr=True, workspace=None, out=None, stre
     """
     torch = _torch()
     f32 = torch.float32
-    if k.dim() != 3:
+    if not _dims(k, "k", 3):
         raise ValueError("k must be (B, T, C)")
     B, T, C = k.shape
     _need(k, "k", f32)
@@ -280,7 +288,7 @@ def wkv_backward_state(w, u, k, v, r, dy, state=None, grad_state=None, want_dr=T
     """
     torch = _torch()
     f32 = torch.float32
-    if k.dim() != 3:
+    if not _dims(k, "k", 3):
         raise ValueError("k must be (B, T, C)")
     B, T, C = k.shape
     _need(k, "k", f32)
@@ -332,7 +340,7 @@ def wkv_forward_checkpointed(w, u, k, v, r=None, state=None, y=None, workspace=N
     """
     torch = _torch()
     f32 = torch.float32
-    if k.dim() != 3:
+    if not _dims(k, "k", 3):
         raise ValueError("k must be (B, T, C)")
     B, T, C = k.shape
     _need(k, "k", f32)
@@ -377,7 +385,7 @@ def wkv7_forward(r, w, k, v, a, b, state=None, y=None, state_out=None, want_stat
     state_out may be given (and may be `state` itself)."""
     torch = _torch()
     f32 = torch.float32
-    if k.dim() != 4:
+    if not _dims(k, "k", 4):
         raise ValueError("k must be (B, T, H, N)")
     B, T, H, N = k.shape
     for n, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b)):
@@ -404,7 +412,7 @@ def wkv_mstate_forward(r, w, k, v, state=None, y=None, state_out=None, want_stat
     (y, S_T), or (y, None) with want_state=False. state_out may be `state` itself."""
     torch = _torch()
     f32 = torch.float32
-    if k.dim() != 4:
+    if not _dims(k, "k", 4):
         raise ValueError("k must be (B, T, H, N)")
     B, T, H, N = k.shape
     for n, t in (("r", r), ("w", w), ("k", k), ("v", v)):
